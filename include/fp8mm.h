@@ -1,0 +1,186 @@
+/*
+ * fp8mm.h -- C ABI of the B200 (sm_100a) scaled FP8 GEMM library (libfp8mm.so).
+ *
+ * The library computes the scaled FP8 GEMM at the core of FP8 LLM inference,
+ *     C_bf16 = (A_e4m3 * scale_a) x (B_e4m3 * scale_b),
+ * in the two scale modes of the source pages, together with the bf16 -> E4M3
+ * quantizer of each mode:
+ *   mode 1, per-token / per-channel fp32 scales -- the deep_gemm.fp8_gemm call
+ *           of page "FP8 推理基础设施（五）：从 DeepGEMM 到 vLLM", listing 1
+ *           (A, B, m, n, k, scale_a[m], scale_b[n]); scale = max|x| / 448 as
+ *           in listing 3 (_calibrate_scales).
+ *   mode 2, MXFP8 1x32 block scales along K with UE8M0 exponents -- the
+ *           mm_mxfp8 path of page "[sglang] FlashInfer v0.6.7 MXFP8 Gemm 통합"
+ *           (section 1: one uint8 scale per 32 elements of K, [n, k // 32];
+ *           section 2: the GEMM call on the quantized activation and the
+ *           pre-processed weight).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named *_bf16, *_e4m3, c, scale*, sf* are DEVICE pointers owned
+ *     by the caller.  The library never allocates, frees or retains device
+ *     memory; it keeps only per-device launch settings.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is enqueued asynchronously on it.  No call syncs the
+ *     host, except fp8mm_last_device_error and fp8mm_selftest_wait_timeout.
+ *   - Matrices are row-major.  A is [m, k] and B is given as [n, k] (the
+ *     transpose of the pages' logical [k, n], K contiguous -- the "weight_t"
+ *     layout of the mm_mxfp8 call).  C is [m, n] bf16 with row stride ldc
+ *     elements.
+ *   - E4M3 is the OCP "fn" variant (max finite 448, no infinities).  Encoding
+ *     rounds to nearest even and saturates to +-448.  bf16 output rounds to
+ *     nearest even.
+ *   - Inputs must be finite; NaN/Inf inputs give unspecified results.
+ *   - Argument errors are returned synchronously, before any CUDA call, so
+ *     they can be checked without a GPU.  A device that is not sm_100 gives
+ *     FP8MM_ERR_UNSUPPORTED.
+ *   - Every wait inside a kernel is bounded.  On expiry the kernel records a
+ *     device error word, frees what it holds and returns.  The host reads the
+ *     word with fp8mm_last_device_error().
+ */
+#ifndef FP8MM_H
+#define FP8MM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int fp8mm_status;
+
+#define FP8MM_OK 0
+#define FP8MM_ERR_NULL 1          /* a required pointer is NULL */
+#define FP8MM_ERR_SHAPE 2         /* negative size, or k not a multiple of the mode's granule */
+#define FP8MM_ERR_ALIGN 3         /* pointer or leading dimension breaks the 16-byte rules */
+#define FP8MM_ERR_UNSUPPORTED 4   /* no sm_100 device current */
+#define FP8MM_ERR_LAUNCH 5        /* a CUDA call failed (the CUDA error is in fp8mm_last_cuda_error) */
+#define FP8MM_ERR_WORKSPACE 6     /* split-K requested without a large enough workspace */
+#define FP8MM_ERR_DEVICE 7        /* a kernel recorded a device-side error (bounded wait expired) */
+
+/* Optional knobs of the GEMM calls (pass NULL for defaults). */
+typedef struct fp8mm_opts {
+  /* Device scratch for the small-M split-K kernel: fp32 partial tiles plus one
+   * 32-bit arrival counter per output tile.  Caller-owned.  It must be zeroed
+   * once before first use (e.g. cudaMemsetAsync); every successful call leaves
+   * the counters zero again.  After a call that reported FP8MM_ERR_DEVICE it
+   * must be zeroed again.  Calls sharing one workspace must not overlap on
+   * the GPU.  NULL disables split-K. */
+  void* workspace;
+  size_t workspace_bytes;
+  /* Kernel choice: FP8MM_KERNEL_AUTO, FP8MM_KERNEL_TILED (persistent 128x256
+   * tiles) or FP8MM_KERNEL_SMALL_M (weights on the MMA M side, tokens on N;
+   * mxfp8_gemm only, m <= 64). */
+  int32_t kernel;
+  /* Number of CTAs for the small-M kernel's stream-K split (0 = one per SM). */
+  int32_t small_m_ctas;
+} fp8mm_opts;
+
+#define FP8MM_KERNEL_AUTO 0
+#define FP8MM_KERNEL_TILED 1
+#define FP8MM_KERNEL_SMALL_M 2
+
+/* ---------------------------------------------------------------- mode 1 */
+
+/* Per-row E4M3 quantizer (mode 1) -- page "从 DeepGEMM 到 vLLM", listing 3
+ * (scale = max|x| / 448) applied per row, feeding listing 1's per-token
+ * scale_a (rows of A) and per-channel scale_b (rows of B^T).
+ *   x_bf16  [rows, k] bf16, row stride ld_x elements
+ *   q_e4m3  [rows, k] E4M3 bytes out, row stride ld_q bytes
+ *   scale   [rows] fp32 out: s[r] = amax_r / 448 (IEEE fp32 division), 1.0 for
+ *           an all-zero row
+ *   q[r, j] = E4M3_RNE_sat(x[r, j] / s[r]) with an IEEE fp32 quotient.
+ * Requires k % 8 == 0, ld_x % 8 == 0, ld_q % 8 == 0, ld_x >= k, ld_q >= k,
+ * x 16-byte aligned, q 8-byte aligned, scale 4-byte aligned.
+ * rows == 0 is a no-op; k == 0 writes scale = 1. */
+fp8mm_status fp8_quantize_rowwise(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x,
+                                  void* q_e4m3, int64_t ld_q, float* scale, void* stream);
+
+/* Per-token / per-channel scaled FP8 GEMM (mode 1) -- deep_gemm.fp8_gemm of
+ * page "从 DeepGEMM 到 vLLM", listing 1.
+ *   c[i, j] = bf16_RNE( scale_a[i] * scale_b[j] * sum_k dec(a[i,k]) dec(b[j,k]) )
+ * with fp32 accumulation on the tensor cores.
+ *   a [m, k] E4M3 (row stride k bytes), b [n, k] E4M3 (row stride k bytes),
+ *   scale_a [m] fp32, scale_b [n] fp32, c [m, n] bf16 with row stride ldc.
+ * Requires k % 16 == 0, a/b 16-byte aligned, c 2-byte aligned, ldc >= n (rows
+ * whose address is 16-byte aligned are written with 16-byte stores).
+ * m == 0 or n == 0 is a no-op; k == 0 writes zeros.  opt may be NULL. */
+fp8mm_status fp8_gemm(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t n, int64_t k,
+                      const float* scale_a, const float* scale_b, void* c_bf16, int64_t ldc,
+                      const fp8mm_opts* opt, void* stream);
+
+/* ---------------------------------------------------------------- mode 2 */
+
+/* Scale-factor (SF) layout of this library.  Rows are padded to a multiple of
+ * 128 and K-blocks (32 elements each) to a multiple of 4.  The buffer is made
+ * of 512-byte chunks, one per (128-row tile rt, group of 4 K-blocks kc),
+ * ordered rt-major: chunk (rt, kc) starts at (rt * n_kc + kc) * 512 with
+ * n_kc = ceil(k / 128).  Inside a chunk, the byte of row r and block b is
+ *     (r % 32) * 16 + ((r % 128) / 32) * 4 + (b % 4),
+ * i.e. each 32-bit word holds the 4 block exponents of one row and each 16-byte
+ * line holds rows r, r+32, r+64, r+96 -- the shape one tcgen05.cp (32x128b,
+ * warpx4) moves into tensor memory.  Padding bytes are written as 0.
+ * Byte value e encodes the scale 2^(e - 127) (UE8M0). */
+size_t fp8mm_sf_bytes(int64_t rows, int64_t k);
+/* Byte offset of (row, block) in that layout; -1 when out of range. */
+int64_t fp8mm_sf_offset(int64_t rows, int64_t k, int64_t row, int64_t block);
+/* Host-memory permutations between that layout and the canonical row-major
+ * [rows, k/32] scale tensor of the pages ([n, k // 32]).  Both pointers are
+ * HOST pointers; nothing is launched. */
+fp8mm_status fp8mm_sf_to_canonical(const uint8_t* sf, int64_t rows, int64_t k, uint8_t* canonical);
+fp8mm_status fp8mm_sf_from_canonical(const uint8_t* canonical, int64_t rows, int64_t k, uint8_t* sf);
+
+/* MXFP8 quantizer (mode 2) -- one UE8M0 exponent per 32 elements of K as in
+ * page "[sglang] FlashInfer v0.6.7 MXFP8 Gemm 통합", section 1, with the
+ * amax/448 rule of page "从 DeepGEMM 到 vLLM", listing 3, restricted to powers
+ * of two:  e = clamp(ceil(log2(amax / 448)) + 127, 0, 254)  (e = 127 for an
+ * all-zero block), q = E4M3_RNE_sat(x * 2^(127 - e)) (the scaling is exact).
+ *   x_bf16 [rows, k] bf16, row stride ld_x; q_e4m3 [rows, k], row stride ld_q;
+ *   sf     fp8mm_sf_bytes(rows, k) bytes in the layout above (written whole,
+ *          padding included).
+ * Requires k % 32 == 0, ld_x % 8 == 0, ld_q % 8 == 0, x 16-byte aligned,
+ * q 8-byte aligned, sf 16-byte aligned.  rows == 0 or k == 0 is a no-op. */
+fp8mm_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, void* q_e4m3,
+                            int64_t ld_q, uint8_t* sf, void* stream);
+
+/* MXFP8 block-scaled GEMM (mode 2) -- the mm_mxfp8(a, b_t, a_sf, b_sf,
+ * out_dtype=bf16) call of page "[sglang] FlashInfer v0.6.7 MXFP8 Gemm 통합",
+ * section 2, with the scales consumed inside the tensor-core MMA:
+ *   c[i, j] = bf16_RNE( sum_b 2^(ea[i,b]-127) 2^(eb[j,b]-127) sum_{k in b} dec(a) dec(b) )
+ *   a [m, k], sf_a fp8mm_sf_bytes(m, k); b [n, k], sf_b fp8mm_sf_bytes(n, k);
+ *   c [m, n] bf16, row stride ldc.
+ * Requires k % 32 == 0, a/b/sf 16-byte aligned, c 2-byte aligned, ldc >= n.
+ * With m <= 64 the small-M (decode) kernel runs: weights b fill the MMA's
+ * 128-row side, tokens the N side, and K is split stream-K style over the SMs
+ * when opt->workspace is given (see fp8mm_workspace_bytes); partial sums are
+ * reduced deterministically (fixed order) by the last CTA of each tile. */
+fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e4m3, const uint8_t* sf_b,
+                        int64_t m, int64_t n, int64_t k, void* c_bf16, int64_t ldc, const fp8mm_opts* opt,
+                        void* stream);
+
+/* Workspace bytes the small-M kernel needs for this shape with `ctas` CTAs
+ * (0 = one per SM of the current device; on a host without a GPU, 148). */
+size_t fp8mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas);
+
+/* ---------------------------------------------------------------- misc */
+
+const char* fp8mm_status_str(fp8mm_status status);
+/* CUDA error code of the last failed CUDA call made by the library (0 if none). */
+int fp8mm_last_cuda_error(void);
+/* Synchronizes the current device, returns the device error word (0 = none;
+ * bits 0-7 kind (1 = bounded wait expired), 8-15 wait site, 16-31 CTA) and
+ * clears it. */
+unsigned int fp8mm_last_device_error(void);
+/* Self-test of the bounded wait: launches one CTA that waits on an mbarrier
+ * nothing will ever arrive at, with a limit of timeout_us microseconds, and
+ * returns after it.  Returns FP8MM_ERR_DEVICE when the wait expired and was
+ * reported as it should be (and clears the word), FP8MM_OK if it unexpectedly
+ * completed. */
+fp8mm_status fp8mm_selftest_wait_timeout(uint32_t timeout_us, void* stream);
+/* ABI version of this header: major * 10000 + minor * 100 + patch. */
+int fp8mm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP8MM_H */

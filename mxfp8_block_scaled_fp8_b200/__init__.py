@@ -1,0 +1,12 @@
+"""B200-native scaled FP8 / MXFP8 GEMM and quantizers (sm_100a).
+
+The compute lives in ``libfp8mm.so`` (hand-written CUDA: tcgen05 / TMA / TMEM
+GEMMs and vectorised quantizers) behind the C ABI of ``include/fp8mm.h``;
+``fp8mm`` is its thin Python binding and ``synthetic`` draws the seeded
+workload inputs.
+"""
+from .fp8mm import (  # noqa: F401
+    Fp8mmError, KERNEL_AUTO, KERNEL_SMALL_M, KERNEL_TILED, fp8_gemm, fp8_quantize_rowwise, last_device_error,
+    mxfp8_gemm, mxfp8_quantize, selftest_wait_timeout, sf_bytes, sf_from_canonical, sf_offset, sf_to_canonical,
+    version, workspace_bytes,
+)

@@ -1,0 +1,308 @@
+// decode.cuh -- small-M (decode) MXFP8 GEMM: C[m, n] for m <= 64 tokens.
+//
+// The arithmetic is the block-scaled GEMM of page "[sglang] FlashInfer v0.6.7
+// MXFP8 Gemm 통합", section 2, with the operand roles swapped: the weight B
+// ([n, k], pre-quantized with its scales) fills the MMA's 128-row M side and
+// the m tokens the N side (padded to kNM = 16..64), so D = B_tile x A^T lands
+// in TMEM as 128 weight rows x kNM tokens.  At these sizes the call is bound
+// by streaming the weight bytes from HBM, so the K range of the n/128 weight
+// tiles is split stream-K style over (up to) one CTA per SM: CTA b owns units
+// [b*U/G, (b+1)*U/G) of the U = n_tiles * num_k (tile, 128-wide K slab)
+// units.  A tile covered by one CTA is written directly; otherwise each
+// contributor stores its fp32 partial in the workspace, bumps the tile's
+// arrival counter, and the last to arrive sums the partials in CTA order
+// (a fixed order, so results do not depend on timing), writes bf16 and
+// resets the counter.  No CTA ever waits for another.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace fp8mm {
+
+constexpr int kDecThreads = 192;
+
+struct DecodeArgs {
+  int m, n, k;
+  int num_k;          // ceil(k / 128)
+  int n_tiles;        // ceil(n / 128)
+  int64_t units;      // n_tiles * num_k
+  int ctas;           // G
+  __nv_bfloat16* c;
+  int64_t ldc;
+  const uint8_t* sfw;  // scales of the weight b (rows = n)
+  const uint8_t* sfx;  // scales of the activation a (rows = m)
+  int n_kc;            // ceil(k / 128)
+  float* partials;     // [2 * G][kNM][128] fp32
+  unsigned* tickets;   // [n_tiles], zero between calls
+  uint64_t timeout_ns;
+};
+
+template <int kNM, int kStages>
+struct DecodeCfg {
+  static_assert(kNM % 16 == 0 && kNM >= 16 && kNM <= 64, "token tile");
+  static constexpr int kWBytes = 128 * 128;
+  static constexpr int kXBytes = kNM * 128;
+  static constexpr int kOffW = 0;
+  static constexpr int kOffX = kOffW + kStages * kWBytes;
+  static constexpr int kOffSfw = kOffX + kStages * kXBytes;
+  static constexpr int kOffSfx = kOffSfw + kStages * 512;
+  static constexpr int kOffBar = kOffSfx + kStages * 512;
+  static constexpr int kNumBars = 2 * kStages + 2 * 2 + 2;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static constexpr int kSfCol0 = 2 * kNM;
+  static constexpr int kColsUsed = kSfCol0 + 8 * kStages;
+  static constexpr int kTmemCols = kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128 : kColsUsed <= 256 ? 256 : 512;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ int64_t dec_unit_start(int b, const DecodeArgs& p) {
+  return static_cast<int64_t>(b) * p.units / p.ctas;
+}
+// CTA that owns unit u: the largest b with floor(b*U/G) <= u.
+__device__ __forceinline__ int dec_owner(int64_t u, const DecodeArgs& p) {
+  return static_cast<int>(((u + 1) * p.ctas - 1) / p.units);
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void regs_fence_16(uint32_t* r) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]));
+}
+
+template <int kNM, int kStages>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                        const DecodeArgs p) {
+  using Cfg = DecodeCfg<kNM, kStages>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint64_t* epi_sync = drain + 1;  // the four epilogue warps meet here (bounded)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.x;
+  const int64_t u_begin = dec_unit_start(b, p);
+  const int64_t u_end = dec_unit_start(b + 1, p);
+  const int first_tile = static_cast<int>(u_begin / p.num_k);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    mbar_init(drain, 1);
+    mbar_init(epi_sync, 4);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int64_t u = u_begin; ok && u < u_end;) {
+        const int t = static_cast<int>(u / p.num_k);
+        const int kb0 = static_cast<int>(u % p.num_k);
+        const int kb1 = static_cast<int>(kb0 + (u_end - u) < p.num_k ? kb0 + (u_end - u) : p.num_k);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], Cfg::kWBytes + Cfg::kXBytes + 1024u);
+          tma_load_2d(smem + Cfg::kOffW + stage * Cfg::kWBytes, &tmW, &full[stage], kb * 128, t * 128);
+          tma_load_2d(smem + Cfg::kOffX + stage * Cfg::kXBytes, &tmX, &full[stage], kb * 128, 0);
+          bulk_load(smem + Cfg::kOffSfw + stage * 512, p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u,
+                    &full[stage]);
+          bulk_load(smem + Cfg::kOffSfx + stage * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[stage]);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        u += kb1 - kb0;
+      }
+      for (int s = 0; s < kStages; ++s)
+        if (issued_mask & (1u << s))
+          mbar_wait(&full[s], (issued_parity >> s) & 1u, p.timeout_ns, nullptr, kSiteProducerDrain);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int64_t u = u_begin; ok && u < u_end;) {
+        const int kb0 = static_cast<int>(u % p.num_k);
+        const int kb1 = static_cast<int>(kb0 + (u_end - u) < p.num_k ? kb0 + (u_end - u) : p.num_k);
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, kSiteMmaAccEmpty)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kNM);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfw_t = tmem_base + static_cast<uint32_t>(Cfg::kSfCol0 + stage * 8);
+          const uint32_t sfx_t = sfw_t + 4u;
+          tmem_cp_32x128b_warpx4(sfw_t, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfw + stage * 512)));
+          tmem_cp_32x128b_warpx4(sfx_t, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfx + stage * 512)));
+          const uint64_t wdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffW + stage * Cfg::kWBytes));
+          const uint64_t xdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffX + stage * Cfg::kXBytes));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_mxf8f6f4(d_tmem, wdesc + 2u * kk, xdesc + 2u * kk, idesc_mxf8f6f4(128, kNM, kk, kk), sfw_t, sfx_t,
+                         (kb != kb0) || (kk != 0));
+          tc_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+        u += kb1 - kb0;
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, p.timeout_ns, nullptr, kSiteDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------ epilogue
+    const int sp = warp & 3;
+    const int nl = sp * 32 + lane;  // weight row inside the tile = output column
+    int acc = 0;
+    uint32_t acc_phase = 0, sync_phase = 0;
+    // All four epilogue warps meet; false if the wait expired or the CTA aborted.
+    auto epi_meet = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_sync);
+      const bool ok = mbar_wait(epi_sync, sync_phase, p.timeout_ns, abort_flag, kSiteEpiSync);
+      sync_phase ^= 1u;
+      return ok;
+    };
+    for (int64_t u = u_begin; u < u_end;) {
+      const int t = static_cast<int>(u / p.num_k);
+      const int kb0 = static_cast<int>(u % p.num_k);
+      const int kb1 = static_cast<int>(kb0 + (u_end - u) < p.num_k ? kb0 + (u_end - u) : p.num_k);
+      u += kb1 - kb0;
+      if (!mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns, abort_flag, kSiteEpiAccFull)) break;
+      tc_fence_after();
+      uint32_t r[kNM];
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(acc * kNM);
+#pragma unroll
+      for (int ch = 0; ch < kNM / 16; ++ch) tmem_ld_32x32b_x16(t_row + ch * 16, r + ch * 16);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int ch = 0; ch < kNM / 16; ++ch) regs_fence_16(r + ch * 16);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+
+      const int n_col = t * 128 + nl;
+      if (kb0 == 0 && kb1 == p.num_k) {
+        if (n_col < p.n) {
+#pragma unroll
+          for (int j = 0; j < kNM; ++j)
+            if (j < p.m) p.c[static_cast<int64_t>(j) * p.ldc + n_col] = __float2bfloat16_rn(__uint_as_float(r[j]));
+        }
+        continue;
+      }
+      // partial tile: publish, count, and let the last contributor reduce
+      const int slot = 2 * b + (t == first_tile ? 0 : 1);
+      float* mine = p.partials + static_cast<int64_t>(slot) * kNM * 128;
+#pragma unroll
+      for (int j = 0; j < kNM; ++j)
+        if (j < p.m) mine[j * 128 + nl] = __uint_as_float(r[j]);
+      __threadfence();
+      if (!epi_meet()) break;
+      const int b_first = dec_owner(static_cast<int64_t>(t) * p.num_k, p);
+      const int b_last = dec_owner(static_cast<int64_t>(t + 1) * p.num_k - 1, p);
+      if (threadIdx.x == 64) {
+        const unsigned prev = atomicAdd(&p.tickets[t], 1u);
+        *last_flag = (prev == static_cast<unsigned>(b_last - b_first)) ? 1 : 0;
+      }
+      if (!epi_meet()) break;
+      if (*last_flag) {
+        __threadfence();
+        float sum[kNM];
+#pragma unroll
+        for (int j = 0; j < kNM; ++j) sum[j] = 0.f;
+        for (int bb = b_first; bb <= b_last; ++bb) {
+          const int first_bb = static_cast<int>(dec_unit_start(bb, p) / p.num_k);
+          const int sl = 2 * bb + (t == first_bb ? 0 : 1);
+          const float* src = p.partials + static_cast<int64_t>(sl) * kNM * 128;
+#pragma unroll
+          for (int j = 0; j < kNM; ++j)
+            if (j < p.m) sum[j] += __ldcg(src + j * 128 + nl);
+        }
+        if (n_col < p.n) {
+#pragma unroll
+          for (int j = 0; j < kNM; ++j)
+            if (j < p.m) p.c[static_cast<int64_t>(j) * p.ldc + n_col] = __float2bfloat16_rn(sum[j]);
+        }
+        if (threadIdx.x == 64) p.tickets[t] = 0u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace fp8mm

@@ -1,0 +1,449 @@
+// fp8mm.cu -- the C ABI of include/fp8mm.h: argument checks, TMA descriptors,
+// launch geometry, and the kernels of quant.cuh / gemm.cuh / decode.cuh
+// (one translation unit, so the device error word is a single symbol).
+#include "fp8mm.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "decode.cuh"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+
+namespace fp8mm {
+
+// ------------------------------------------------------------------ host state
+static thread_local int t_last_cuda_error = 0;
+
+static fp8mm_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return FP8MM_ERR_LAUNCH;
+}
+
+struct DeviceInfo {
+  int device = -1;
+  int sms = 0;
+  bool sm100 = false;
+};
+
+static std::mutex g_mu;
+
+static fp8mm_status current_device(DeviceInfo* info) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  static DeviceInfo cache[64];
+  if (dev < 0 || dev >= 64) return FP8MM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (cache[dev].device != dev) {
+    int major = 0, sms = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    cache[dev].device = dev;
+    cache[dev].sms = sms;
+    cache[dev].sm100 = (major == 10);
+  }
+  *info = cache[dev];
+  return info->sm100 ? FP8MM_OK : FP8MM_ERR_UNSUPPORTED;
+}
+
+// Opt a kernel into its dynamic shared memory size, once per device.
+static fp8mm_status ensure_smem(const void* kernel, int bytes, int dev) {
+  static std::set<std::pair<const void*, int>> done;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (done.count({kernel, dev})) return FP8MM_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e);
+  done.insert({kernel, dev});
+  return FP8MM_OK;
+}
+
+static uint64_t wait_timeout_ns() {
+  static uint64_t ns = [] {
+    const char* s = std::getenv("FP8MM_WAIT_TIMEOUT_MS");
+    long long ms = s ? std::atoll(s) : 0;
+    return static_cast<uint64_t>(ms > 0 ? ms : 2000) * 1000000ull;
+  }();
+  return ns;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major uint8 matrix [rows, k] (row stride k bytes),
+// box = 128 bytes of K x box_rows rows, 128-byte swizzle, zero fill outside.
+static fp8mm_status make_map(CUtensorMap* map, const void* base, int64_t k, int64_t rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};
+  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return FP8MM_OK;
+}
+
+static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+static fp8mm_status launched() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FP8MM_OK : cuda_fail(e);
+}
+
+// ------------------------------------------------------------------ kernels' configs
+using G1 = GemmCfg<false, 256, 4, 2>;
+using G2 = GemmCfg<true, 256, 4, 1>;
+constexpr int kDecStages = 8;
+
+__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the wait must expire and report.
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, timeout_ns, &abort_flag, kSiteSelfTest);
+}
+
+// ------------------------------------------------------------------ launchers
+static fp8mm_status launch_tiled(bool mx, const void* a, const void* b, const uint8_t* sfa, const uint8_t* sfb,
+                                 int64_t m, int64_t n, int64_t k, const float* sa, const float* sb, void* c,
+                                 int64_t ldc, cudaStream_t stream, const DeviceInfo& dev) {
+  CUtensorMap ta, tb;
+  fp8mm_status st = make_map(&ta, a, k, m, kBM);
+  if (st != FP8MM_OK) return st;
+  st = make_map(&tb, b, k, n, 256);
+  if (st != FP8MM_OK) return st;
+  GemmArgs p{};
+  p.m = static_cast<int>(m);
+  p.n = static_cast<int>(n);
+  p.k = static_cast<int>(k);
+  p.num_k = static_cast<int>(cdiv(k, kBK));
+  p.tiles_m = static_cast<int>(cdiv(m, kBM));
+  p.tiles_n = static_cast<int>(cdiv(n, 256));
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.c = static_cast<__nv_bfloat16*>(c);
+  p.ldc = ldc;
+  p.sa = sa;
+  p.sb = sb;
+  p.sfa = sfa;
+  p.sfb = sfb;
+  p.n_kc = static_cast<int>(cdiv(k, 128));
+  p.sfb_row_tiles = static_cast<int>(cdiv(n, 128));
+  p.timeout_ns = wait_timeout_ns();
+  const int grid = std::min(p.num_tiles, dev.sms);
+  if (mx) {
+    auto kern = gemm_tiled_kernel<true, 256, 4, 1>;
+    if ((st = ensure_smem(reinterpret_cast<const void*>(kern), G2::kSmemBytes, dev.device)) != FP8MM_OK) return st;
+    kern<<<grid, kGemmThreads, G2::kSmemBytes, stream>>>(ta, tb, p);
+  } else {
+    auto kern = gemm_tiled_kernel<false, 256, 4, 2>;
+    if ((st = ensure_smem(reinterpret_cast<const void*>(kern), G1::kSmemBytes, dev.device)) != FP8MM_OK) return st;
+    kern<<<grid, kGemmThreads, G1::kSmemBytes, stream>>>(ta, tb, p);
+  }
+  return launched();
+}
+
+static int small_m_tile(int64_t m) { return m <= 16 ? 16 : m <= 32 ? 32 : m <= 48 ? 48 : 64; }
+
+static size_t small_m_partials_bytes(int ctas, int nm) {
+  size_t b = static_cast<size_t>(2) * ctas * nm * 128 * sizeof(float);
+  return (b + 255) & ~size_t(255);
+}
+
+template <int kNM>
+static fp8mm_status launch_small_m_t(const CUtensorMap& tw, const CUtensorMap& tx, const DecodeArgs& p,
+                                     cudaStream_t stream, int dev) {
+  using Cfg = DecodeCfg<kNM, kDecStages>;
+  auto kern = gemm_small_m_kernel<kNM, kDecStages>;
+  fp8mm_status st = ensure_smem(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, dev);
+  if (st != FP8MM_OK) return st;
+  kern<<<p.ctas, kDecThreads, Cfg::kSmemBytes, stream>>>(tw, tx, p);
+  return launched();
+}
+
+static fp8mm_status launch_small_m(const void* a, const uint8_t* sfa, const void* b, const uint8_t* sfb, int64_t m,
+                                   int64_t n, int64_t k, void* c, int64_t ldc, const fp8mm_opts* opt,
+                                   cudaStream_t stream, const DeviceInfo& dev) {
+  const int nm = small_m_tile(m);
+  DecodeArgs p{};
+  p.m = static_cast<int>(m);
+  p.n = static_cast<int>(n);
+  p.k = static_cast<int>(k);
+  p.num_k = static_cast<int>(cdiv(k, 128));
+  p.n_tiles = static_cast<int>(cdiv(n, 128));
+  p.units = static_cast<int64_t>(p.n_tiles) * p.num_k;
+  p.c = static_cast<__nv_bfloat16*>(c);
+  p.ldc = ldc;
+  p.sfw = sfb;
+  p.sfx = sfa;
+  p.n_kc = p.num_k;
+  p.timeout_ns = wait_timeout_ns();
+  if (opt == nullptr || opt->workspace == nullptr) {
+    p.ctas = p.n_tiles;  // one CTA per weight tile, whole K: no partial sums
+  } else {
+    int64_t g = opt->small_m_ctas > 0 ? opt->small_m_ctas : dev.sms;
+    g = std::min<int64_t>(g, p.units);
+    p.ctas = static_cast<int>(std::max<int64_t>(g, 1));
+    const size_t need = fp8mm_workspace_bytes(m, n, k, p.ctas);
+    if (opt->workspace_bytes < need || !aligned(opt->workspace, 256)) return FP8MM_ERR_WORKSPACE;
+    p.partials = static_cast<float*>(opt->workspace);
+    p.tickets = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(opt->workspace) +
+                                            small_m_partials_bytes(p.ctas, nm));
+  }
+  CUtensorMap tw, tx;
+  fp8mm_status st = make_map(&tw, b, k, n, 128);
+  if (st != FP8MM_OK) return st;
+  st = make_map(&tx, a, k, m, nm);
+  if (st != FP8MM_OK) return st;
+  switch (nm) {
+    case 16: return launch_small_m_t<16>(tw, tx, p, stream, dev.device);
+    case 32: return launch_small_m_t<32>(tw, tx, p, stream, dev.device);
+    case 48: return launch_small_m_t<48>(tw, tx, p, stream, dev.device);
+    default: return launch_small_m_t<64>(tw, tx, p, stream, dev.device);
+  }
+}
+
+}  // namespace fp8mm
+
+using namespace fp8mm;
+
+// ====================================================================== C ABI
+extern "C" {
+
+int fp8mm_version(void) { return 10000; }
+
+const char* fp8mm_status_str(fp8mm_status s) {
+  switch (s) {
+    case FP8MM_OK: return "ok";
+    case FP8MM_ERR_NULL: return "null pointer";
+    case FP8MM_ERR_SHAPE: return "bad shape";
+    case FP8MM_ERR_ALIGN: return "misaligned pointer or leading dimension";
+    case FP8MM_ERR_UNSUPPORTED: return "no sm_100 device";
+    case FP8MM_ERR_LAUNCH: return "CUDA call failed";
+    case FP8MM_ERR_WORKSPACE: return "workspace missing or too small";
+    case FP8MM_ERR_DEVICE: return "device-side error (bounded wait expired)";
+    default: return "unknown status";
+  }
+}
+
+int fp8mm_last_cuda_error(void) { return t_last_cuda_error; }
+
+size_t fp8mm_sf_bytes(int64_t rows, int64_t k) {
+  if (rows <= 0 || k <= 0) return 0;
+  return static_cast<size_t>(cdiv(rows, 128) * 128) * static_cast<size_t>(cdiv(k, 128)) * 4;
+}
+
+int64_t fp8mm_sf_offset(int64_t rows, int64_t k, int64_t row, int64_t block) {
+  if (rows <= 0 || k <= 0) return -1;
+  const int64_t n_kc = cdiv(k, 128);
+  if (row < 0 || row >= cdiv(rows, 128) * 128 || block < 0 || block >= n_kc * 4) return -1;
+  return ((row / 128) * n_kc + block / 4) * 512 + (row % 32) * 16 + ((row % 128) / 32) * 4 + (block % 4);
+}
+
+fp8mm_status fp8mm_sf_to_canonical(const uint8_t* sf, int64_t rows, int64_t k, uint8_t* canonical) {
+  if (rows < 0 || k < 0 || k % 32 != 0) return FP8MM_ERR_SHAPE;
+  if (rows == 0 || k == 0) return FP8MM_OK;
+  if (sf == nullptr || canonical == nullptr) return FP8MM_ERR_NULL;
+  const int64_t nkb = k / 32;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < nkb; ++b) canonical[r * nkb + b] = sf[fp8mm_sf_offset(rows, k, r, b)];
+  return FP8MM_OK;
+}
+
+fp8mm_status fp8mm_sf_from_canonical(const uint8_t* canonical, int64_t rows, int64_t k, uint8_t* sf) {
+  if (rows < 0 || k < 0 || k % 32 != 0) return FP8MM_ERR_SHAPE;
+  if (rows == 0 || k == 0) return FP8MM_OK;
+  if (sf == nullptr || canonical == nullptr) return FP8MM_ERR_NULL;
+  std::memset(sf, 0, fp8mm_sf_bytes(rows, k));
+  const int64_t nkb = k / 32;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < nkb; ++b) sf[fp8mm_sf_offset(rows, k, r, b)] = canonical[r * nkb + b];
+  return FP8MM_OK;
+}
+
+size_t fp8mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas) {
+  if (m <= 0 || n <= 0 || k <= 0 || m > 64) return 0;
+  int g = ctas;
+  if (g <= 0) {
+    int dev = 0, sms = 0;
+    g = (cudaGetDevice(&dev) == cudaSuccess &&
+         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+            ? sms
+            : 148;
+    cudaGetLastError();  // a host without a GPU leaves an error behind
+  }
+  const int64_t units = cdiv(n, 128) * cdiv(k, 128);
+  g = static_cast<int>(std::min<int64_t>(g, units));
+  const size_t tickets = static_cast<size_t>(cdiv(n, 128)) * sizeof(unsigned);
+  return small_m_partials_bytes(g, small_m_tile(m)) + ((tickets + 255) & ~size_t(255));
+}
+
+fp8mm_status fp8_quantize_rowwise(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, void* q_e4m3,
+                                  int64_t ld_q, float* scale, void* stream) {
+  if (rows < 0 || k < 0 || k % 8 != 0) return FP8MM_ERR_SHAPE;
+  if (rows == 0) return FP8MM_OK;
+  if (scale == nullptr) return FP8MM_ERR_NULL;
+  if (!aligned(scale, 4)) return FP8MM_ERR_ALIGN;
+  if (k > 0) {  // with k == 0 only the scales are written (x and q are not touched)
+    if (ld_x < k || ld_q < k) return FP8MM_ERR_SHAPE;
+    if (x_bf16 == nullptr || q_e4m3 == nullptr) return FP8MM_ERR_NULL;
+    if (!aligned(x_bf16, 16) || !aligned(q_e4m3, 8) || ld_x % 8 != 0 || ld_q % 8 != 0) return FP8MM_ERR_ALIGN;
+  }
+  DeviceInfo dev;
+  fp8mm_status st = current_device(&dev);
+  if (st != FP8MM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const auto* x = static_cast<const __nv_bfloat16*>(x_bf16);
+  auto* q = static_cast<uint8_t*>(q_e4m3);
+  const int64_t nvec = k / 8;
+  if (nvec > static_cast<int64_t>(kQ1Threads) * 8) {
+    const int grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(dev.sms) * 8));
+    quant_rowwise_2pass_kernel<<<grid, kQ1Threads, 0, s>>>(x, rows, k, ld_x, q, ld_q, scale);
+    return launched();
+  }
+  const int threads = static_cast<int>(std::min<int64_t>(kQ1Threads, std::max<int64_t>(32, cdiv(nvec, 32) * 32)));
+  const int64_t nv = cdiv(std::max<int64_t>(nvec, 1), threads);
+  const int per_sm = 2048 / threads;
+  const int grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(dev.sms) * per_sm));
+  if (nv <= 1)
+    quant_rowwise_kernel<1><<<grid, threads, 0, s>>>(x, rows, k, ld_x, q, ld_q, scale);
+  else if (nv <= 2)
+    quant_rowwise_kernel<2><<<grid, threads, 0, s>>>(x, rows, k, ld_x, q, ld_q, scale);
+  else if (nv <= 4)
+    quant_rowwise_kernel<4><<<grid, threads, 0, s>>>(x, rows, k, ld_x, q, ld_q, scale);
+  else
+    quant_rowwise_kernel<8><<<grid, threads, 0, s>>>(x, rows, k, ld_x, q, ld_q, scale);
+  return launched();
+}
+
+fp8mm_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, void* q_e4m3, int64_t ld_q,
+                            uint8_t* sf, void* stream) {
+  if (rows < 0 || k < 0 || k % 32 != 0 || ld_x < k || ld_q < k) return FP8MM_ERR_SHAPE;
+  if (rows == 0 || k == 0) return FP8MM_OK;
+  if (x_bf16 == nullptr || q_e4m3 == nullptr || sf == nullptr) return FP8MM_ERR_NULL;
+  if (!aligned(x_bf16, 16) || !aligned(q_e4m3, 8) || !aligned(sf, 16) || ld_x % 8 != 0 || ld_q % 8 != 0)
+    return FP8MM_ERR_ALIGN;
+  DeviceInfo dev;
+  fp8mm_status st = current_device(&dev);
+  if (st != FP8MM_OK) return st;
+  const int64_t n_kc = cdiv(k, 128);
+  const int64_t n_groups = cdiv(rows, 128) * 128 * n_kc;
+  const int64_t groups_per_cta_step = (kQ2Threads / 32) * 2;
+  const int64_t want = cdiv(n_groups, groups_per_cta_step * kQ2Unroll);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(dev.sms) * 8)));
+  quant_mx_kernel<<<grid, kQ2Threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x_bf16), rows, k, ld_x, static_cast<uint8_t*>(q_e4m3), ld_q, sf, n_kc,
+      n_groups);
+  return launched();
+}
+
+static fp8mm_status check_gemm_common(const void* a, const void* b, int64_t m, int64_t n, int64_t k, const void* c,
+                                      int64_t ldc, int64_t k_granule) {
+  if (m < 0 || n < 0 || k < 0 || k % k_granule != 0 || ldc < n) return FP8MM_ERR_SHAPE;
+  if (m > INT32_MAX / 2 || n > INT32_MAX / 2 || k > INT32_MAX / 2) return FP8MM_ERR_SHAPE;
+  if (m == 0 || n == 0) return FP8MM_OK;
+  if (c == nullptr || (k > 0 && (a == nullptr || b == nullptr))) return FP8MM_ERR_NULL;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(c, 2)) return FP8MM_ERR_ALIGN;
+  return FP8MM_OK;
+}
+
+static fp8mm_status zero_output(void* c, int64_t m, int64_t n, int64_t ldc, cudaStream_t s) {
+  cudaError_t e = cudaMemset2DAsync(c, static_cast<size_t>(ldc) * 2, 0, static_cast<size_t>(n) * 2,
+                                    static_cast<size_t>(m), s);
+  return e == cudaSuccess ? FP8MM_OK : cuda_fail(e);
+}
+
+fp8mm_status fp8_gemm(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t n, int64_t k, const float* scale_a,
+                      const float* scale_b, void* c_bf16, int64_t ldc, const fp8mm_opts* opt, void* stream) {
+  fp8mm_status st = check_gemm_common(a_e4m3, b_e4m3, m, n, k, c_bf16, ldc, 16);
+  if (st != FP8MM_OK || m == 0 || n == 0) return st;
+  if (k > 0 && (scale_a == nullptr || scale_b == nullptr)) return FP8MM_ERR_NULL;
+  if (!aligned(scale_a, 4) || !aligned(scale_b, 4)) return FP8MM_ERR_ALIGN;
+  if (opt != nullptr && opt->kernel == FP8MM_KERNEL_SMALL_M) return FP8MM_ERR_SHAPE;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != FP8MM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (k == 0) return zero_output(c_bf16, m, n, ldc, s);
+  return launch_tiled(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev);
+}
+
+fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e4m3, const uint8_t* sf_b, int64_t m,
+                        int64_t n, int64_t k, void* c_bf16, int64_t ldc, const fp8mm_opts* opt, void* stream) {
+  fp8mm_status st = check_gemm_common(a_e4m3, b_e4m3, m, n, k, c_bf16, ldc, 32);
+  if (st != FP8MM_OK || m == 0 || n == 0) return st;
+  if (k > 0 && (sf_a == nullptr || sf_b == nullptr)) return FP8MM_ERR_NULL;
+  if (!aligned(sf_a, 16) || !aligned(sf_b, 16)) return FP8MM_ERR_ALIGN;
+  const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
+  if (kind == FP8MM_KERNEL_SMALL_M && m > 64) return FP8MM_ERR_SHAPE;
+  if (kind < FP8MM_KERNEL_AUTO || kind > FP8MM_KERNEL_SMALL_M) return FP8MM_ERR_SHAPE;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != FP8MM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (k == 0) return zero_output(c_bf16, m, n, ldc, s);
+  const bool small = (kind == FP8MM_KERNEL_SMALL_M) || (kind == FP8MM_KERNEL_AUTO && m <= 64);
+  if (small) return launch_small_m(a_e4m3, sf_a, b_e4m3, sf_b, m, n, k, c_bf16, ldc, opt, s, dev);
+  return launch_tiled(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev);
+}
+
+unsigned int fp8mm_last_device_error(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    t_last_cuda_error = static_cast<int>(e);
+    return 0xFFFFFFFFu;
+  }
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
+  const unsigned int zero = 0;
+  cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  return v;
+}
+
+fp8mm_status fp8mm_selftest_wait_timeout(uint32_t timeout_us, void* stream) {
+  DeviceInfo dev;
+  fp8mm_status st = current_device(&dev);
+  if (st != FP8MM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  selftest_wait_kernel<<<1, 32, 0, s>>>(static_cast<uint64_t>(timeout_us) * 1000ull);
+  if ((st = launched()) != FP8MM_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const unsigned int word = fp8mm_last_device_error();
+  if (word == 0xFFFFFFFFu) return FP8MM_ERR_LAUNCH;
+  return ((word & 0xFFu) == kDevErrTimeout && ((word >> 8) & 0xFFu) == kSiteSelfTest) ? FP8MM_ERR_DEVICE
+                                                                                          : FP8MM_OK;
+}
+
+}  // extern "C"

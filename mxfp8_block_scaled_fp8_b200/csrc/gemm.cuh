@@ -1,0 +1,303 @@
+// gemm.cuh -- persistent, warp-specialised tcgen05 GEMM for both scale modes.
+//
+//   mode 1: C = diag(scale_a) (A x B^T) diag(scale_b)  (page "从 DeepGEMM 到
+//           vLLM", listing 1: fp8_gemm with per-token scale_a[m] and
+//           per-channel scale_b[n]); kind::f8f6f4, scales applied in the
+//           epilogue in fp32.
+//   mode 2: C = sum over 32-wide K blocks of 2^(ea-127) 2^(eb-127) A_b B_b^T
+//           (page "[sglang] FlashInfer v0.6.7 MXFP8 Gemm 통합", section 2,
+//           mm_mxfp8); kind::mxf8f6f4.block_scale, scales consumed by the MMA
+//           from TMEM.
+//
+// One CTA per SM loops over 128 x kBN output tiles (grouped raster: kGroupM
+// M-tiles share each B tile while it is hot in L2).  Warp roles:
+//   warp 0      TMA producer: A/B tiles (128-byte swizzle) and, in mode 2,
+//               the 512-byte scale chunks, into a kStages-deep ring.
+//   warp 1      allocates TMEM; one lane issues tcgen05.mma (and tcgen05.cp of
+//               the scale chunks) per 128-byte K slab, commits to free the slab.
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (each warp owns
+//               the 32 TMEM lanes of its sub-partition), scaling, bf16 RNE,
+//               stores.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace fp8mm {
+
+constexpr int kBM = 128;            // tile rows (A / M side of the MMA)
+constexpr int kBK = 128;            // K elements (= bytes) per pipeline slab
+constexpr int kMmaK = 32;           // K per tcgen05.mma for 8-bit operands
+constexpr int kGemmThreads = 192;   // 6 warps
+constexpr int kGroupM = 16;
+
+struct GemmArgs {
+  int m, n, k;
+  int num_k;                 // ceil(k / kBK)
+  int tiles_m, tiles_n, num_tiles;
+  __nv_bfloat16* c;
+  int64_t ldc;
+  const float* sa;           // mode 1
+  const float* sb;
+  const uint8_t* sfa;        // mode 2 (library scale layout)
+  const uint8_t* sfb;
+  int n_kc;                  // scale chunks per 128-row tile = ceil(k / 128)
+  int sfb_row_tiles;         // ceil(n / 128): 128-row tiles present in sfb
+  uint64_t timeout_ns;
+};
+
+template <bool kMX, int kBN, int kStages, int kAccStages>
+struct GemmCfg {
+  static_assert(kBN % 128 == 0 && kBN <= 256, "B tile rows");
+  static constexpr int kABytes = kBM * kBK;
+  static constexpr int kBBytes = kBN * kBK;
+  static constexpr int kSfaBytes = kMX ? 512 : 0;
+  static constexpr int kSfbChunks = kBN / 128;
+  static constexpr int kSfbBytes = kMX ? kSfbChunks * 512 : 0;
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + kStages * kABytes;
+  static constexpr int kOffSfa = kOffB + kStages * kBBytes;
+  static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
+  static constexpr int kOffBar = kOffSfb + kStages * kSfbBytes;
+  static constexpr int kNumBars = 2 * kStages + 2 * kAccStages + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack to align the base to 1024
+  // TMEM columns: accumulators, then (mode 2) per-stage scale columns:
+  // 4 for the A chunk, 4 per 128 rows of B.
+  static constexpr int kSfColsPerStage = 4 + 4 * kSfbChunks;
+  static constexpr int kSfCol0 = kAccStages * kBN;
+  static constexpr int kColsUsed = kSfCol0 + (kMX ? kStages * kSfColsPerStage : 0);
+  static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
+                                   : kColsUsed <= 256 ? 256 : 512;
+  static_assert(kColsUsed <= 512, "TMEM budget");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ void tile_coords(int t, const GemmArgs& p, int& mb, int& nb) {
+  const int per_group = kGroupM * p.tiles_n;
+  const int g = t / per_group;
+  const int first_m = g * kGroupM;
+  const int gm = min(p.tiles_m - first_m, kGroupM);
+  const int r = t - g * per_group;
+  mb = first_m + r % gm;
+  nb = r / gm;
+}
+
+template <bool kMX, int kBN, int kStages, int kAccStages>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const GemmArgs p) {
+  using Cfg = GemmCfg<kMX, kBN, kStages, kAccStages>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + kAccStages;
+  uint64_t* drain = acc_empty + kAccStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < kAccStages; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(t, p, mb, nb);
+        int sfb_chunks = 0;
+        if constexpr (kMX) sfb_chunks = min(Cfg::kSfbChunks, p.sfb_row_tiles - nb * Cfg::kSfbChunks);
+        for (int kb = 0; kb < p.num_k; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) {
+            ok = false;
+            break;
+          }
+          uint32_t bytes = Cfg::kABytes + Cfg::kBBytes;
+          if constexpr (kMX) bytes += 512u + 512u * sfb_chunks;
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_2d(smem + Cfg::kOffA + stage * Cfg::kABytes, &tmA, &full[stage], kb * kBK, mb * kBM);
+          tma_load_2d(smem + Cfg::kOffB + stage * Cfg::kBBytes, &tmB, &full[stage], kb * kBK, nb * kBN);
+          if constexpr (kMX) {
+            bulk_load(smem + Cfg::kOffSfa + stage * 512, p.sfa + (static_cast<int64_t>(mb) * p.n_kc + kb) * 512,
+                      512u, &full[stage]);
+            for (int i = 0; i < sfb_chunks; ++i)
+              bulk_load(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes + i * 512,
+                        p.sfb + (static_cast<int64_t>(nb * Cfg::kSfbChunks + i) * p.n_kc + kb) * 512, 512u,
+                        &full[stage]);
+          }
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Let every copy this thread started land before the CTA can exit.
+      for (int s = 0; s < kStages; ++s)
+        if (issued_mask & (1u << s))
+          mbar_wait(&full[s], (issued_parity >> s) & 1u, p.timeout_ns, nullptr, kSiteProducerDrain);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, kSiteMmaAccEmpty)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+        for (int kb = 0; kb < p.num_k; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffA + stage * Cfg::kABytes));
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffB + stage * Cfg::kBBytes));
+          if constexpr (kMX) {
+            const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(Cfg::kSfCol0 + stage * Cfg::kSfColsPerStage);
+            const uint32_t sfb_t = sfa_t + 4u;
+            tmem_cp_32x128b_warpx4(sfa_t, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfa + stage * 512)));
+#pragma unroll
+            for (int i = 0; i < Cfg::kSfbChunks; ++i)
+              tmem_cp_32x128b_warpx4(sfb_t + 4u * i,
+                                     sf_chunk_desc(smem_u32(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes + i * 512)));
+#pragma unroll
+            for (int kk = 0; kk < kBK / kMmaK; ++kk)
+              mma_mxf8f6f4(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8f6f4(kBM, kBN, kk, kk), sfa_t, sfb_t,
+                           (kb | kk) != 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kBK / kMmaK; ++kk)
+              mma_f8f6f4(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_f8f6f4(kBM, kBN), (kb | kk) != 0);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);
+        if (++acc == kAccStages) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // Every MMA / copy this thread issued must finish before TMEM is freed.
+      tc_commit(drain);
+      mbar_wait(drain, 0, p.timeout_ns, nullptr, kSiteDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------ epilogue
+    const int sp = warp & 3;  // TMEM sub-partition this warp can read
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+      int mb, nb;
+      tile_coords(t, p, mb, nb);
+      if (!mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns, abort_flag, kSiteEpiAccFull)) break;
+      tc_fence_after();
+      const int row = mb * kBM + sp * 32 + lane;
+      float s_row = 1.f;
+      if constexpr (!kMX) s_row = (row < p.m) ? __ldg(p.sa + row) : 0.f;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(acc * kBN);
+#pragma unroll 1
+      for (int ch = 0; ch < kBN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + ch * 32, r);
+        tmem_ld_wait_32(r);
+        if (ch == kBN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        }
+        const int col0 = nb * kBN + ch * 32;
+        float sbv = 1.f;
+        if constexpr (!kMX) sbv = (col0 + lane < p.n) ? __ldg(p.sb + col0 + lane) : 0.f;
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float v0 = __uint_as_float(r[2 * j]);
+          float v1 = __uint_as_float(r[2 * j + 1]);
+          if constexpr (!kMX) {
+            v0 = v0 * s_row * __shfl_sync(0xFFFFFFFFu, sbv, 2 * j);
+            v1 = v1 * s_row * __shfl_sync(0xFFFFFFFFu, sbv, 2 * j + 1);
+          }
+          __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+          packed[j] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        if (row < p.m && col0 < p.n) {
+          __nv_bfloat16* dst = p.c + static_cast<int64_t>(row) * p.ldc + col0;
+          if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              *reinterpret_cast<uint4*>(dst + q4 * 8) =
+                  make_uint4(packed[4 * q4], packed[4 * q4 + 1], packed[4 * q4 + 2], packed[4 * q4 + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (col0 + j < p.n) {
+                const uint32_t w = packed[j >> 1];
+                *reinterpret_cast<uint16_t*>(dst + j) = static_cast<uint16_t>((j & 1) ? (w >> 16) : (w & 0xFFFFu));
+              }
+            }
+          }
+        }
+      }
+      if (++acc == kAccStages) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace fp8mm

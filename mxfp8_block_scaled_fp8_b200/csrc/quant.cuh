@@ -1,0 +1,232 @@
+// quant.cuh -- bf16 -> E4M3 quantizers for both scale modes (HBM-bound).
+//
+// Mode 1 (per row):  s = amax / 448 (IEEE fp32 division, 1 for a zero row),
+//   q = E4M3_RNE_sat(x / s).  Page "从 DeepGEMM 到 vLLM", listing 3
+//   (_calibrate_scales) applied per row; listing 1 takes per-token scale_a
+//   and per-channel scale_b.
+// Mode 2 (MX, 1x32 blocks along K):  e = clamp(ceil(log2(amax/448)) + 127,
+//   0, 254), 127 for a zero block; q = E4M3_RNE_sat(x * 2^(127-e)).  Page
+//   "[sglang] FlashInfer v0.6.7 MXFP8 Gemm 통합", section 1 (one uint8 scale
+//   per 32 elements).
+//
+// Both kernels read bf16 with 16-byte vector loads and write E4M3 with
+// 8-byte stores; a warp always covers a contiguous run of one row.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cstdint>
+
+namespace fp8mm {
+
+__device__ __forceinline__ uint4 ld_stream_16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// The 8 bf16 values of a 16-byte vector as fp32 (exact).
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ float absmax8(const float (&f)[8]) {
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+  return m;
+}
+
+// 8 fp32 -> 8 E4M3 bytes (round to nearest even, saturate to +-448), element 0
+// in the lowest byte.
+__device__ __forceinline__ uint2 f32x8_to_e4m3(const float (&y)[8]) {
+  uint32_t b[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    b[i] = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(y[2 * i], y[2 * i + 1]),
+                                                          __NV_SATFINITE, __NV_E4M3));
+  return make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
+}
+
+// ------------------------------------------------------------------ mode 1
+
+constexpr int kQ1Threads = 256;
+
+// One CTA per row (grid-stride over rows).  The row is held in registers
+// (NV 16-byte vectors per thread), so x is read once; rows longer than
+// NV * blockDim * 8 elements use the two-pass variant below.
+template <int NV>
+__global__ void __launch_bounds__(kQ1Threads) quant_rowwise_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                                                   int64_t k, int64_t ld_x, uint8_t* __restrict__ q,
+                                                                   int64_t ld_q, float* __restrict__ scale) {
+  __shared__ float red[kQ1Threads / 32];
+  const int nvec = static_cast<int>(k / 8);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const __nv_bfloat16* xr = x + row * ld_x;
+    uint4 v[NV];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int idx = threadIdx.x + i * blockDim.x;
+      if (idx < nvec) {
+        v[i] = ld_stream_16(xr + static_cast<int64_t>(idx) * 8);
+        float f[8];
+        bf16x8_to_f32(v[i], f);
+        amax = fmaxf(amax, absmax8(f));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    float m = 0.f;
+    const int nw = blockDim.x >> 5;
+    for (int w = 0; w < nw; ++w) m = fmaxf(m, red[w]);
+    __syncthreads();  // red[] is rewritten by the next row
+    const float s = (m == 0.f) ? 1.f : __fdiv_rn(m, 448.f);
+    if (threadIdx.x == 0) scale[row] = s;
+    uint8_t* qr = q + row * ld_q;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int idx = threadIdx.x + i * blockDim.x;
+      if (idx < nvec) {
+        float f[8];
+        bf16x8_to_f32(v[i], f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] = __fdiv_rn(f[j], s);
+        *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(idx) * 8) = f32x8_to_e4m3(f);
+      }
+    }
+  }
+}
+
+// Long rows: one pass for the maximum, a second pass (mostly from L2) to
+// quantize.
+__global__ void __launch_bounds__(kQ1Threads) quant_rowwise_2pass_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                         int64_t rows, int64_t k, int64_t ld_x,
+                                                                         uint8_t* __restrict__ q, int64_t ld_q,
+                                                                         float* __restrict__ scale) {
+  __shared__ float red[kQ1Threads / 32];
+  const int64_t nvec = k / 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const __nv_bfloat16* xr = x + row * ld_x;
+    float amax = 0.f;
+    for (int64_t idx = threadIdx.x; idx < nvec; idx += blockDim.x) {
+      float f[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(xr + idx * 8), f);
+      amax = fmaxf(amax, absmax8(f));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    float m = 0.f;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+    __syncthreads();
+    const float s = (m == 0.f) ? 1.f : __fdiv_rn(m, 448.f);
+    if (threadIdx.x == 0) scale[row] = s;
+    uint8_t* qr = q + row * ld_q;
+    for (int64_t idx = threadIdx.x; idx < nvec; idx += blockDim.x) {
+      float f[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(xr + idx * 8), f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[j] = __fdiv_rn(f[j], s);
+      *reinterpret_cast<uint2*>(qr + idx * 8) = f32x8_to_e4m3(f);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ mode 2
+
+// UE8M0 exponent of a block maximum a (an exact bf16 value held in fp32):
+// a = (1 + m/128) 2^(Ea-127) and 448 = 1.75 * 2^8, so
+// ceil(log2(a/448)) + 127 = Ea - 8 + (m > 96); clamped to [0, 254];
+// a bf16 subnormal gives 0 and a == 0 gives 127.
+__device__ __forceinline__ int mx_exponent(float a) {
+  const uint32_t bits = __float_as_uint(a);
+  const int Ea = static_cast<int>(bits >> 23);
+  const int m7 = static_cast<int>((bits >> 16) & 0x7Fu);
+  if (Ea == 0) return (a == 0.f) ? 127 : 0;
+  const int e = Ea - 8 + (m7 > 96 ? 1 : 0);
+  return e < 0 ? 0 : (e > 254 ? 254 : e);
+}
+
+// 2^(127 - e) as fp32, exactly (e in [0, 254]).
+__device__ __forceinline__ float mx_inv_scale(int e) {
+  return (e < 254) ? __uint_as_float(static_cast<uint32_t>(254 - e) << 23) : __uint_as_float(0x00400000u);
+}
+
+constexpr int kQ2Threads = 256;
+constexpr int kQ2Unroll = 4;
+
+// Work unit ("group") = one row x 4 consecutive K-blocks = 128 elements =
+// 16 lanes x 16 bytes, producing one 32-bit word of the scale layout.  A warp
+// handles two groups per step.  Groups cover the padded scale buffer, so the
+// padding words (rows >= rows, blocks >= k/32) are written as 0 here too.
+__global__ void __launch_bounds__(kQ2Threads) quant_mx_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                                              int64_t k, int64_t ld_x, uint8_t* __restrict__ q,
+                                                              int64_t ld_q, uint8_t* __restrict__ sf, int64_t n_kc,
+                                                              int64_t n_groups) {
+  const int lane = threadIdx.x & 31;
+  const int half = lane >> 4;    // which of the warp's two groups
+  const int sub = lane & 15;     // lane within the group
+  const int kb_in = sub >> 2;    // K-block within the group
+  const int v_in = sub & 3;      // 16-byte vector within the block
+  const int64_t nkb = k / 32;
+  const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t step = nwarps * 2;
+
+  for (int64_t g0 = warp_id * 2; g0 < n_groups; g0 += step * kQ2Unroll) {
+    uint4 v[kQ2Unroll];
+    int64_t row[kQ2Unroll], kb[kQ2Unroll], g[kQ2Unroll];
+    bool real[kQ2Unroll];
+#pragma unroll
+    for (int u = 0; u < kQ2Unroll; ++u) {
+      g[u] = g0 + u * step + half;
+      const int64_t gg = g[u] < n_groups ? g[u] : 0;
+      row[u] = gg / n_kc;
+      kb[u] = (gg % n_kc) * 4 + kb_in;
+      real[u] = (g[u] < n_groups) && (row[u] < rows) && (kb[u] < nkb);
+      v[u] = real[u] ? ld_stream_16(x + row[u] * ld_x + kb[u] * 32 + v_in * 8) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kQ2Unroll; ++u) {
+      float f[8];
+      bf16x8_to_f32(v[u], f);
+      float amax = absmax8(f);
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+      const int e = real[u] ? mx_exponent(amax) : 0;
+      if (real[u]) {
+        const float inv = mx_inv_scale(e);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] *= inv;  // exact: power-of-two scaling
+        *reinterpret_cast<uint2*>(q + row[u] * ld_q + kb[u] * 32 + v_in * 8) = f32x8_to_e4m3(f);
+      }
+      // gather the group's four exponents into its first lane
+      const int base = half * 16;
+      const uint32_t e0 = __shfl_sync(0xFFFFFFFFu, e, base + 0);
+      const uint32_t e1 = __shfl_sync(0xFFFFFFFFu, e, base + 4);
+      const uint32_t e2 = __shfl_sync(0xFFFFFFFFu, e, base + 8);
+      const uint32_t e3 = __shfl_sync(0xFFFFFFFFu, e, base + 12);
+      if (sub == 0 && g[u] < n_groups) {
+        const int64_t r = row[u];
+        const int64_t kc = g[u] % n_kc;
+        const int64_t off = ((r / 128) * n_kc + kc) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4;
+        *reinterpret_cast<uint32_t*>(sf + off) = e0 | (e1 << 8) | (e2 << 16) | (e3 << 24);
+      }
+    }
+  }
+}
+
+}  // namespace fp8mm

@@ -1,0 +1,106 @@
+"""The C-ABI library loads without a GPU, exports every function the header
+declares, rejects bad arguments before touching CUDA, and its host-side scale
+layout helpers agree with the layout formula the header documents."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import mxfp8_block_scaled_fp8_b200 as fp8mm
+from mxfp8_block_scaled_fp8_b200 import fp8mm as binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8mm.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:[A-Za-z_][\w\s\*]*?)\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if not n.startswith("FP8MM")))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(binding.LIB_PATH)
+    declared = _declared()
+    assert {"fp8_quantize_rowwise", "mxfp8_quantize", "fp8_gemm", "mxfp8_gemm"} <= set(declared)
+    missing = [n for n in declared if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(binding._SIGNATURES) <= set(declared) | {"fp8mm_version"}
+
+
+def test_version_and_status_strings():
+    L = binding.lib()
+    assert L.fp8mm_version() == 10000
+    for s in range(0, 8):
+        assert len(L.fp8mm_status_str(s)) > 0
+    assert L.fp8mm_status_str(99) == b"unknown status"
+
+
+def test_argument_errors_without_a_gpu():
+    L = binding.lib()
+    P = ctypes.c_void_p
+    fake = 1 << 20                                             # never dereferenced
+    # shapes
+    assert L.fp8_gemm(P(fake), P(fake), 4, 4, 15, P(fake), P(fake), P(fake), 8, None, None) == 2
+    assert L.mxfp8_gemm(P(fake), P(fake), P(fake), P(fake), 4, 4, 48, P(fake), 8, None, None) == 2
+    assert L.fp8_quantize_rowwise(P(fake), 4, 12, 16, P(fake), 16, P(fake), None) == 2
+    assert L.mxfp8_quantize(P(fake), 4, 40, 40, P(fake), 40, P(fake), None) == 2
+    assert L.fp8_gemm(P(fake), P(fake), -1, 4, 16, P(fake), P(fake), P(fake), 8, None, None) == 2
+    assert L.fp8_gemm(P(fake), P(fake), 4, 16, 16, P(fake), P(fake), P(fake), 8, None, None) == 2   # ldc < n
+    # null pointers
+    assert L.fp8_gemm(None, P(fake), 4, 4, 16, P(fake), P(fake), P(fake), 8, None, None) == 1
+    assert L.mxfp8_gemm(P(fake), None, P(fake), P(fake), 4, 4, 32, P(fake), 8, None, None) == 1
+    assert L.mxfp8_quantize(P(fake), 4, 32, 32, P(fake), 32, None, None) == 1
+    # alignment
+    assert L.fp8_gemm(P(fake + 8), P(fake), 4, 4, 16, P(fake), P(fake), P(fake), 8, None, None) == 3
+    assert L.fp8_gemm(P(fake), P(fake), 4, 4, 16, P(fake), P(fake), P(fake + 1), 12, None, None) == 3
+    assert L.mxfp8_quantize(P(fake), 4, 32, 36, P(fake), 32, P(fake), None) == 3
+    # empty problems are no-ops and need no device
+    assert L.fp8_gemm(None, None, 0, 4, 16, None, None, None, 8, None, None) == 0
+    assert L.mxfp8_quantize(None, 0, 64, 64, None, 64, None, None) == 0
+    assert L.fp8_quantize_rowwise(None, 0, 64, 64, None, 64, None, None) == 0
+
+
+def test_workspace_sizes():
+    # 2 * G * 128 * NM floats (256-byte aligned) + one counter per 128-row tile
+    assert fp8mm.workspace_bytes(64, 14336, 4096, 148) == 2 * 148 * 128 * 64 * 4 + 512
+    assert fp8mm.workspace_bytes(1, 4096, 14336, 148) == 2 * 148 * 128 * 16 * 4 + 256
+    assert fp8mm.workspace_bytes(65, 4096, 4096, 148) == 0            # only for m <= 64
+    assert fp8mm.workspace_bytes(8, 128, 128, 148) == 2 * 1 * 128 * 16 * 4 + 256   # clamped to 1 unit
+
+
+def _layout_offset(rows, k, r, b):
+    n_kc = -(-k // 128)
+    return ((r // 128) * n_kc + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + (b % 4)
+
+
+@pytest.mark.parametrize("rows,k", [(1, 32), (130, 96), (256, 4096), (300, 160)])
+def test_scale_layout_helpers(rows, k):
+    assert fp8mm.sf_bytes(rows, k) == (-(-rows // 128) * 128) * (-(-k // 128)) * 4
+    nkb = k // 32
+    rng = np.random.default_rng(rows + k)
+    canon = rng.integers(0, 255, size=(rows, nkb), dtype=np.uint8)
+    sf = fp8mm.sf_from_canonical(torch.from_numpy(canon), rows, k).numpy()
+    expect = np.zeros(fp8mm.sf_bytes(rows, k), dtype=np.uint8)
+    for r in range(rows):
+        for b in range(nkb):
+            assert fp8mm.sf_offset(rows, k, r, b) == _layout_offset(rows, k, r, b)
+            expect[_layout_offset(rows, k, r, b)] = canon[r, b]
+    assert np.array_equal(sf, expect)
+    assert np.array_equal(fp8mm.sf_to_canonical(torch.from_numpy(sf), rows, k).numpy(), canon)
+    # every byte of the buffer belongs to exactly one (row, block) of the padded grid
+    rp, kb4 = -(-rows // 128) * 128, -(-k // 128) * 4
+    offs = sorted(fp8mm.sf_offset(rows, k, r, b) for r in range(rp) for b in range(kb4))
+    assert offs == list(range(fp8mm.sf_bytes(rows, k)))
+    assert fp8mm.sf_offset(rows, k, rp, 0) == -1
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(binding.Fp8mmError):
+        binding.lib()

@@ -1,0 +1,121 @@
+"""Small-M (decode) MXFP8 kernel vs the CPU oracle: every M in {1, 8, 32, 64}
+against the three Llama-3-8B-sized linears, with and without the stream-K
+split, plus determinism and partition independence."""
+import numpy as np
+import pytest
+import torch
+
+import mxfp8_block_scaled_fp8_b200 as fp8mm
+from mxfp8_block_scaled_fp8_b200 import synthetic
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    gu.require_gpu()
+
+
+@pytest.fixture(scope="module")
+def decode_data():
+    import oracle as orc
+    ws, xs = synthetic.decode()
+    out = {}
+    for name, w in ws.items():
+        qw, sfw = orc.mx_quantize(synthetic.bits(w))
+        gw, gsfw = fp8mm.mxfp8_quantize(gu.to_dev(w))
+        out[name] = (qw, sfw, gw, gsfw)
+    return out, xs
+
+
+def _workspace(m, n, k, ctas=0):
+    nbytes = fp8mm.workspace_bytes(m, n, k, ctas)
+    return torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+
+
+@pytest.mark.parametrize("name", ["up", "down", "qkv"])
+@pytest.mark.parametrize("m", synthetic.DECODE_M)
+def test_decode_sweep_stream_k(decode_data, name, m):
+    import oracle as orc
+    weights, xs = decode_data
+    qw, sfw, gw, gsfw = weights[name]
+    n, k = synthetic.DECODE_SHAPES[name]
+    x = xs[k][:m].contiguous()
+    qx, sfx = orc.mx_quantize(synthetic.bits(x))
+    gx, gsfx = fp8mm.mxfp8_quantize(gu.to_dev(x))
+    ws = _workspace(m, n, k)
+    c = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws)
+    torch.cuda.synchronize()
+    c_ref, bound = orc.gemm_mx(qx, sfx, qw, sfw)
+    gu.check_gemm(c, c_ref, bound, f"decode {name} m={m}")
+    # counters are left at zero for the next call
+    c2 = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(c, c2), "second call with the same workspace differs"
+
+
+@pytest.mark.parametrize("m", [1, 64])
+def test_decode_without_workspace(decode_data, m):
+    import oracle as orc
+    weights, xs = decode_data
+    qw, sfw, gw, gsfw = weights["qkv"]
+    n, k = synthetic.DECODE_SHAPES["qkv"]
+    x = xs[k][:m].contiguous()
+    qx, sfx = orc.mx_quantize(synthetic.bits(x))
+    gx, gsfx = fp8mm.mxfp8_quantize(gu.to_dev(x))
+    c = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw)
+    torch.cuda.synchronize()
+    c_ref, bound = orc.gemm_mx(qx, sfx, qw, sfw)
+    gu.check_gemm(c, c_ref, bound, f"decode qkv m={m} one CTA per tile")
+
+
+@pytest.mark.parametrize("ctas", [1, 7, 37, 300, 5000])
+def test_decode_partitions(decode_data, ctas):
+    """Different stream-K partitions (including more CTAs than units) all meet
+    the bar; each partition is deterministic."""
+    import oracle as orc
+    weights, xs = decode_data
+    qw, sfw, gw, gsfw = weights["down"]
+    n, k = synthetic.DECODE_SHAPES["down"]
+    m = 8
+    x = xs[k][:m].contiguous()
+    qx, sfx = orc.mx_quantize(synthetic.bits(x))
+    gx, gsfx = fp8mm.mxfp8_quantize(gu.to_dev(x))
+    ws = _workspace(m, n, k, ctas)
+    c1 = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, small_m_ctas=ctas)
+    c2 = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, small_m_ctas=ctas)
+    torch.cuda.synchronize()
+    c_ref, bound = orc.gemm_mx(qx, sfx, qw, sfw)
+    gu.check_gemm(c1, c_ref, bound, f"decode down m=8 ctas={ctas}")
+    assert torch.equal(c1, c2)
+
+
+@pytest.mark.parametrize("m,n,k", [(3, 200, 96), (17, 130, 4128), (64, 384, 320), (33, 1000, 64)])
+def test_decode_ragged(m, n, k):
+    import oracle as orc
+    x = synthetic.random_bf16((m, k), seed=m * 3 + k)
+    w = synthetic.random_bf16((n, k), seed=n * 5 + k, sigma=0.02)
+    qx, sfx = orc.mx_quantize(synthetic.bits(x))
+    qw, sfw = orc.mx_quantize(synthetic.bits(w))
+    gx, gsfx = fp8mm.mxfp8_quantize(gu.to_dev(x))
+    gw, gsfw = fp8mm.mxfp8_quantize(gu.to_dev(w))
+    c_ref, bound = orc.gemm_mx(qx, sfx, qw, sfw)
+    for ctas in (0, 5):
+        ws = _workspace(m, n, k, ctas)
+        c = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, small_m_ctas=ctas)
+        torch.cuda.synchronize()
+        gu.check_gemm(c, c_ref, bound, f"decode ragged {m}x{n}x{k} ctas={ctas}")
+    c = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, kernel=fp8mm.KERNEL_TILED)
+    torch.cuda.synchronize()
+    gu.check_gemm(c, c_ref, bound, f"tiled {m}x{n}x{k}")
+
+
+def test_workspace_too_small_is_rejected(decode_data):
+    weights, xs = decode_data
+    _, _, gw, gsfw = weights["qkv"]
+    n, k = synthetic.DECODE_SHAPES["qkv"]
+    gx, gsfx = fp8mm.mxfp8_quantize(gu.to_dev(xs[k][:8].contiguous()))
+    ws = torch.zeros(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fp8mm.Fp8mmError):
+        fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws)

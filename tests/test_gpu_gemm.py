@@ -1,0 +1,170 @@
+"""GPU GEMMs vs the CPU oracle within the acceptance bar
+|c - c_ref| <= 4e-3 sum|a b| + 2^-8 |c_ref| and rel-Fro <= 2e-3.
+
+The oracle side quantizes the same seeded bf16 inputs with the oracle and
+multiplies exactly in fp64; the GPU side runs the library's quantizers and
+GEMMs.  Full-size workloads are checked on sampled rows and columns (the
+oracle computes them one by one)."""
+import numpy as np
+import pytest
+import torch
+
+import mxfp8_block_scaled_fp8_b200 as fp8mm
+from mxfp8_block_scaled_fp8_b200 import synthetic
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    gu.require_gpu()
+
+
+def _rows_cols(m, n, nr, nc, seed):
+    g = np.random.default_rng(seed)
+    rows = np.sort(g.choice(m, size=min(nr, m), replace=False))
+    cols = np.sort(g.choice(n, size=min(nc, n), replace=False))
+    # always include the ragged edges
+    rows = np.unique(np.concatenate([rows, [0, m - 1]]))
+    cols = np.unique(np.concatenate([cols, [0, n - 1]]))
+    return rows, cols
+
+
+def run_rowwise(a_cpu, bt_cpu, sample=None, label=""):
+    """Mode 1 end to end: quantize both operands per row, GEMM, compare."""
+    import oracle as orc
+    qa, sa = orc.quantize_rowwise(synthetic.bits(a_cpu))
+    qb, sb = orc.quantize_rowwise(synthetic.bits(bt_cpu))
+    ga, gsa = fp8mm.fp8_quantize_rowwise(gu.to_dev(a_cpu))
+    gb, gsb = fp8mm.fp8_quantize_rowwise(gu.to_dev(bt_cpu))
+    c = fp8mm.fp8_gemm(ga, gb, gsa, gsb)
+    torch.cuda.synchronize()
+    if sample is None:
+        c_ref, bound = orc.gemm_rowwise(qa, qb, sa, sb)
+        return gu.check_gemm(c, c_ref, bound, label)
+    rows, cols = sample
+    c_ref, bound = orc.gemm_rowwise(qa[rows], qb, sa[rows], sb)
+    gu.check_gemm(c[torch.from_numpy(rows).cuda()], c_ref, bound, label + " rows")
+    c_ref, bound = orc.gemm_rowwise(qa, qb[cols], sa, sb[cols])
+    gu.check_gemm(c[:, torch.from_numpy(cols).cuda()], c_ref, bound, label + " cols")
+
+
+def run_mx(a_cpu, bt_cpu, sample=None, label="", **kw):
+    """Mode 2 end to end: block-quantize both operands, GEMM, compare."""
+    import oracle as orc
+    qa, sfa = orc.mx_quantize(synthetic.bits(a_cpu))
+    qb, sfb = orc.mx_quantize(synthetic.bits(bt_cpu))
+    ga, gsfa = fp8mm.mxfp8_quantize(gu.to_dev(a_cpu))
+    gb, gsfb = fp8mm.mxfp8_quantize(gu.to_dev(bt_cpu))
+    c = fp8mm.mxfp8_gemm(ga, gsfa, gb, gsfb, **kw)
+    torch.cuda.synchronize()
+    if sample is None:
+        c_ref, bound = orc.gemm_mx(qa, sfa, qb, sfb)
+        return gu.check_gemm(c, c_ref, bound, label)
+    rows, cols = sample
+    c_ref, bound = orc.gemm_mx(qa[rows], sfa[rows], qb, sfb)
+    gu.check_gemm(c[torch.from_numpy(rows).cuda()], c_ref, bound, label + " rows")
+    c_ref, bound = orc.gemm_mx(qa, sfa, qb[cols], sfb[cols])
+    gu.check_gemm(c[:, torch.from_numpy(cols).cuda()], c_ref, bound, label + " cols")
+
+
+# ------------------------------------------------------------ workloads
+
+def test_tiny_rowwise_full():
+    a, bt = synthetic.tiny()
+    run_rowwise(a, bt, label="tiny 128x256x512")
+
+
+def test_qk_mx_full():
+    a, bt = synthetic.qk()
+    run_mx(a, bt, label="qk 2048x1024x4096", kernel=fp8mm.KERNEL_TILED)
+
+
+def test_attn_rowwise_sampled():
+    a, bt = synthetic.attn()
+    run_rowwise(a, bt, sample=_rows_cols(8192, 2048, 192, 64, 2), label="attn 8192x2048x8192")
+
+
+def test_ffn_up_mx_sampled():
+    x, w = synthetic.ffn_up()
+    run_mx(x, w, sample=_rows_cols(8192, 22016, 96, 96, 3), label="ffn_up 8192x22016x8192")
+
+
+# ------------------------------------------------------------ shapes and edges
+
+@pytest.mark.parametrize("m,n,k", [(1, 256, 512), (200, 136, 320), (129, 257, 160), (256, 512, 16),
+                                   (300, 1000, 1040), (128, 256, 128)])
+def test_rowwise_ragged(m, n, k):
+    a = synthetic.random_bf16((m, k), seed=m + 1)
+    bt = synthetic.random_bf16((n, k), seed=n + 2)
+    run_rowwise(a, bt, label=f"rowwise {m}x{n}x{k}")
+
+
+@pytest.mark.parametrize("m,n,k", [(65, 256, 512), (200, 136, 320), (129, 257, 96), (300, 1000, 1056),
+                                   (128, 128, 32), (1, 384, 256)])
+def test_mx_ragged_tiled(m, n, k):
+    a = synthetic.random_bf16((m, k), seed=m + 3)
+    bt = synthetic.random_bf16((n, k), seed=n + 4, sigma=0.05)
+    run_mx(a, bt, label=f"mx {m}x{n}x{k}", kernel=fp8mm.KERNEL_TILED)
+
+
+def test_unit_scales_selection_closed_form():
+    """Listing 1's call shape with scale_a = ones(m), scale_b = ones(n): A selects
+    rows of B exactly, so C equals decoded B rows (exactly representable)."""
+    import oracle as orc
+    m, n, k = 128, 256, 512
+    rng = np.random.default_rng(0)
+    qb = rng.integers(0, 256, size=(n, k), dtype=np.uint8)
+    qb[(qb & 0x7F) == 0x7F] = 0x38
+    qa = np.zeros((m, k), dtype=np.uint8)
+    pick = rng.integers(0, k, size=m)
+    qa[np.arange(m), pick] = 0x38              # 1.0
+    ones_m, ones_n = np.ones(m, np.float32), np.ones(n, np.float32)
+    c = fp8mm.fp8_gemm(torch.from_numpy(qa).cuda(), torch.from_numpy(qb).cuda(), torch.from_numpy(ones_m).cuda(),
+                       torch.from_numpy(ones_n).cuda())
+    c_ref, bound = orc.gemm_rowwise(qa, qb, ones_m, ones_n)
+    dec = orc.e4m3_decode_table()
+    assert np.array_equal(c_ref, dec[qb[:, pick].T])
+    gu.check_gemm(c, c_ref, bound, "selection")
+    assert np.array_equal(c.float().cpu().numpy(), c_ref.astype(np.float32))
+
+
+def test_k_zero_and_empty():
+    a = torch.empty((4, 0), dtype=torch.uint8, device="cuda")
+    b = torch.empty((8, 0), dtype=torch.uint8, device="cuda")
+    c = torch.full((4, 8), 7.0, dtype=torch.bfloat16, device="cuda")
+    sa = torch.ones(4, device="cuda")
+    sb = torch.ones(8, device="cuda")
+    fp8mm.fp8_gemm(a, b, sa, sb, c=c)
+    torch.cuda.synchronize()
+    assert torch.all(c == 0)
+    e = torch.empty((0, 64), dtype=torch.uint8, device="cuda")
+    fp8mm.fp8_gemm(e, torch.zeros((8, 64), dtype=torch.uint8, device="cuda"), sa[:0], sb)
+
+
+def test_strided_output():
+    a = synthetic.random_bf16((130, 256), seed=9)
+    bt = synthetic.random_bf16((200, 256), seed=10)
+    import oracle as orc
+    qa, sa = orc.quantize_rowwise(synthetic.bits(a))
+    qb, sb = orc.quantize_rowwise(synthetic.bits(bt))
+    ga, gsa = fp8mm.fp8_quantize_rowwise(gu.to_dev(a))
+    gb, gsb = fp8mm.fp8_quantize_rowwise(gu.to_dev(bt))
+    big = torch.full((130, 264), 3.0, dtype=torch.bfloat16, device="cuda")
+    fp8mm.fp8_gemm(ga, gb, gsa, gsb, c=big[:, :200])
+    torch.cuda.synchronize()
+    c_ref, bound = orc.gemm_rowwise(qa, qb, sa, sb)
+    gu.check_gemm(big[:, :200], c_ref, bound, "strided c")
+    assert torch.all(big[:, 200:] == 3.0)       # nothing written past n
+
+
+def test_repeat_calls_bit_identical():
+    a, bt = synthetic.tiny()
+    ga, gsa = fp8mm.fp8_quantize_rowwise(gu.to_dev(a))
+    gb, gsb = fp8mm.fp8_quantize_rowwise(gu.to_dev(bt))
+    c1 = fp8mm.fp8_gemm(ga, gb, gsa, gsb)
+    c2 = fp8mm.fp8_gemm(ga, gb, gsa, gsb)
+    torch.cuda.synchronize()
+    assert torch.equal(c1, c2)
+    assert fp8mm.last_device_error() == 0
