@@ -1,0 +1,453 @@
+"""Benchmark of the scaled FP8 GEMM hot path on B200.
+
+Headline workload (one "step" = the whole per-call hot path on one batch):
+  ffn_up: X bf16 [8192, 8192] -> mxfp8_quantize -> mxfp8_gemm against the
+  pre-quantized W [22016, 8192] (MXFP8, 1x32 UE8M0 blocks) -> C bf16.
+  This is the FFN up-projection shape of the "从 DeepGEMM 到 vLLM" page's
+  benchmark_gemm listing, and the largest single-GPU configuration.
+  value = 2*M*N*K per step / step time, in TFLOPS.
+
+The other hot-path rows (per-row quantizer, rowwise GEMM, Q.K^T MX GEMM,
+the decode sweep) are measured in the "rows" object of the same JSON line.
+
+Multi-GPU (torchrun): every rank runs its own replica on its own GPU (no
+data-path collective; weak scaling); time = max over ranks.
+
+--impl reference: the CPU oracle as it stands, on a bounded sample of the
+same workload, on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP8 GEMM TFLOPS & % of B200 FP8 peak; quantize/decode GB/s & % of HBM"
+M, N, K = 8192, 22016, 8192
+FLOPS_PER_STEP = 2.0 * M * N * K
+CPU_SAMPLE_ROWS = 256        # cpu_baseline: this many full rows of C
+REF_ROWS_PER_STEP = 16       # reference arm: a 16 x 2752 block of C per step
+REF_COLS_PER_STEP = N // 8
+
+
+# ---------------------------------------------------------------- helpers
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def _src_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "mxfp8_block_scaled_fp8_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t[kernel_key]
+        return e["bytes_per_launch"] if e.get("src_hash") == _src_hash() else None
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {"gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+               "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100}
+
+    def __init__(self, index: int, period_s: float = 0.01, pci_bus_id: str | None = None):
+        self.index, self.period, self.pci = index, period_s, pci_bus_id
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = None
+            if self.pci:
+                try:
+                    self._h = pynvml.nvmlDeviceGetHandleByPciBusId(self.pci)
+                except Exception:
+                    self._h = None
+            if self._h is None:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception:
+            self._nv = None
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Largest value over all ranks (the slowest rank sets the job time)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank runs `steps` steps of its own replica."""
+    return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------- GPU timing utilities
+
+def _timed(fn, reps, warmup, flush=None, stream=None):
+    """Median device time (ms) of fn over reps, CUDA events on the launching
+    stream, L2 flushed (outside the events) before each rep when given."""
+    import torch
+    s = stream or torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    times = []
+    for _ in range(reps):
+        if flush is not None:
+            flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        fn()
+        b.record(s)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times), min(times)
+
+
+def _rows_measurements(fp8mm, synthetic, peaks, reps=20):
+    """Per-row measurements of the other hot-path steps (each its own unit)."""
+    import torch
+    dev = torch.device("cuda")
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = lambda: flush_buf.zero_()
+    out = {}
+    hbm = peaks["hbm_gbs"]
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+
+    # per-row quantizer and rowwise GEMM on the attention-like workload
+    a, bt = synthetic.attn()
+    a, bt = a.to(dev), bt.to(dev)
+    qa = torch.empty(a.shape, dtype=torch.uint8, device=dev)
+    sa = torch.empty(a.shape[0], dtype=torch.float32, device=dev)
+    t, _ = _timed(lambda: fp8mm.fp8_quantize_rowwise(a, qa, sa), reps, 3, flush)
+    R, Kq = a.shape
+    gbs = (3.0 * R * Kq + 4 * R) / (t * 1e-3) / 1e9
+    out["quantize_rowwise_8192x8192"] = {"ms": t, "GB/s": gbs, "frac_hbm": gbs / hbm}
+    qb, sb = fp8mm.fp8_quantize_rowwise(bt)
+    c = torch.empty((a.shape[0], bt.shape[0]), dtype=torch.bfloat16, device=dev)
+    t, _ = _timed(lambda: fp8mm.fp8_gemm(qa, qb, sa, sb, c), reps, 3, flush)
+    tf = 2.0 * 8192 * 2048 * 8192 / (t * 1e-3) / 1e12
+    out["fp8_gemm_8192x2048x8192"] = {"ms": t, "TFLOPS": tf, "frac_fp8_peak": tf / fp8_peak}
+    del a, bt, qa, qb, c
+
+    # MX Q.K^T shape (64 output tiles: fewer than the 148 SMs)
+    a, bt = synthetic.qk()
+    qa, sfa = fp8mm.mxfp8_quantize(a.to(dev))
+    qb, sfb = fp8mm.mxfp8_quantize(bt.to(dev))
+    c = torch.empty((2048, 1024), dtype=torch.bfloat16, device=dev)
+    t, _ = _timed(lambda: fp8mm.mxfp8_gemm(qa, sfa, qb, sfb, c), reps, 3, flush)
+    tf = 2.0 * 2048 * 1024 * 4096 / (t * 1e-3) / 1e12
+    out["mxfp8_gemm_2048x1024x4096"] = {"ms": t, "TFLOPS": tf, "frac_fp8_peak": tf / fp8_peak}
+
+    # MX quantizer on the FFN weight (done once at load) -- measured standalone
+    _, w = synthetic.ffn_up()
+    w = w.to(dev)
+    qw = torch.empty(w.shape, dtype=torch.uint8, device=dev)
+    sfw = torch.empty(fp8mm.sf_bytes(*w.shape), dtype=torch.uint8, device=dev)
+    t, _ = _timed(lambda: fp8mm.mxfp8_quantize(w, qw, sfw), reps, 3, flush)
+    R, Kq = w.shape
+    gbs = (3.0 * R * Kq + R * Kq / 32) / (t * 1e-3) / 1e9
+    out["mxfp8_quantize_22016x8192"] = {"ms": t, "GB/s": gbs, "frac_hbm": gbs / hbm}
+    del w, qw, sfw
+
+    # decode sweep: quantize X per call + small-M GEMM against a resident weight
+    ws_, xs = synthetic.decode()
+    sweep = {}
+    for name, w in ws_.items():
+        n, k = synthetic.DECODE_SHAPES[name]
+        qw, sfw = fp8mm.mxfp8_quantize(w.to(dev))
+        for m in synthetic.DECODE_M:
+            x = xs[k][:m].contiguous().to(dev)
+            qx = torch.empty((m, k), dtype=torch.uint8, device=dev)
+            sfx = torch.empty(fp8mm.sf_bytes(m, k), dtype=torch.uint8, device=dev)
+            c = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+            wsp = torch.zeros(fp8mm.workspace_bytes(m, n, k), dtype=torch.uint8, device=dev)
+
+            def call():
+                fp8mm.mxfp8_quantize(x, qx, sfx)
+                fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c, workspace=wsp)
+            t, _ = _timed(call, reps, 3, flush)
+            tg, _ = _timed(lambda: fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c, workspace=wsp), reps, 3, flush)
+            e2e_bytes = n * k + n * k / 32 + 2 * m * k + 2 * m * n
+            gemm_bytes = n * k + n * k / 32 + m * k + 128 * k / 32 + 2 * m * n
+            sweep[f"{name}_{n}x{k}_m{m}"] = {
+                "ms": t, "GB/s": e2e_bytes / (t * 1e-3) / 1e9, "frac_hbm": e2e_bytes / (t * 1e-3) / 1e9 / hbm,
+                "gemm_ms": tg, "gemm_GB/s": gemm_bytes / (tg * 1e-3) / 1e9}
+    out["decode"] = sweep
+    return out
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import mxfp8_block_scaled_fp8_b200 as fp8mm
+    from mxfp8_block_scaled_fp8_b200 import synthetic
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+    peaks = _peaks()
+
+    x_cpu, w_cpu = synthetic.ffn_up()
+    x = x_cpu.to(dev)
+    w = w_cpu.to(dev)
+    qw, sfw = fp8mm.mxfp8_quantize(w)              # weights quantized once, at load
+    del w
+    qx = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    sfx = torch.empty(fp8mm.sf_bytes(M, K), dtype=torch.uint8, device=dev)
+    c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fp8mm.mxfp8_quantize(x, qx, sfx)
+        fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    pci = None
+    if hasattr(props, "pci_bus_id"):
+        pci = f"{getattr(props, 'pci_domain_id', 0):08X}:{props.pci_bus_id:02X}:{getattr(props, 'pci_device_id', 0):02X}.0"
+    with ClockSampler(local, pci_bus_id=pci) as clocks:
+        t_start.record(stream)
+        for e0, e1, e2 in evs:
+            e0.record(stream)
+            fp8mm.mxfp8_quantize(x, qx, sfx)
+            e1.record(stream)
+            fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c)
+            e2.record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    q_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in evs) / args.steps
+    g_ms = sum(e1.elapsed_time(e2) for _, e1, e2 in evs) / args.steps
+    total_ms = max_over_ranks(total_ms, dev)
+    ms_per_step = total_ms / args.steps
+    value = job_tflops(FLOPS_PER_STEP, args.steps, ws, total_ms)
+
+    # end to end through the public API with host buffers: H2D of X, the two
+    # calls, D2H of C, all inside the timed region
+    x_host = x_cpu.pin_memory()
+    c_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(2, min(args.steps, 5))
+    for _ in range(2):
+        x.copy_(x_host, non_blocking=True)
+        step()
+        c_host.copy_(c, non_blocking=True)
+    torch.cuda.synchronize()
+    a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_ev.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(x_host, non_blocking=True)
+        step()
+        c_host.copy_(c, non_blocking=True)
+    b_ev.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a_ev.elapsed_time(b_ev) / e2e_steps
+    e2e_ms = max_over_ranks(e2e_ms, dev)
+
+    rows = None
+    if rank == 0 and not args.no_rows:
+        rows = _rows_measurements(fp8mm, synthetic, peaks)
+
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    achieved = FLOPS_PER_STEP / (g_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": ws, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3", "data": "synthetic (seeded N(0,1) X, N(0,0.02^2) W, 0.1% x20 outliers)",
+        "config": {"workload": "ffn_up: X [8192,8192] bf16 -> mxfp8_quantize -> mxfp8_gemm with W [22016,8192] "
+                               "pre-quantized MXFP8 (1x32 UE8M0), bf16 out",
+                   "M": M, "N": N, "K": K, "parallelism": f"dp{ws} (independent replicas)",
+                   "l2": "inputs larger than L2: X 128 MiB bf16 and Wq 172 MiB are re-read every step"},
+        "e2e": {"value": job_tflops(FLOPS_PER_STEP, 1, ws, e2e_ms), "unit": "TFLOPS",
+                "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": c_host.numel() * 2,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "kernels": {"mxfp8_quantize_ms": q_ms, "mxfp8_gemm_ms": g_ms},
+        "roofline": {"bound": "tensor", "kernel": "gemm_tiled_kernel<mx> (mxfp8_gemm)", "achieved": achieved,
+                     "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
+                     "traffic": _ncu_traffic("mxfp8_gemm_ffn_up"),
+                     "peak_note": f"FP8 dense = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s "
+                                  f"(nominal FP8/BF16 ratio); sustained-based peak "
+                                  f"{2.0 * peaks['bf16_tflops_sustained']:.0f}",
+                     "algorithmic": "2*M*N*K flops per launch"},
+        "quantize_roofline": {"bound": "hbm", "achieved": (3.0 * M * K + M * K / 32) / (q_ms * 1e-3) / 1e9,
+                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": (3.0 * M * K + M * K / 32) / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                              "traffic": _ncu_traffic("mxfp8_quantize_x")},
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(CPU_SAMPLE_ROWS, _oracle_workload(x_cpu, w_cpu))
+    if rows is not None:
+        line["rows"] = rows
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def _oracle_workload(x=None, w=None):
+    import oracle
+    from mxfp8_block_scaled_fp8_b200 import synthetic
+    if x is None:
+        x, w = synthetic.ffn_up()
+    qw, sfw = oracle.mx_quantize(synthetic.bits(w))   # weights quantized once (untimed, as on the GPU)
+    return oracle, synthetic, x, qw, sfw
+
+
+def _oracle_step(oracle, synthetic, x, qw, sfw, r0, rows, c0=0, cols=N):
+    qx, sfx = oracle.mx_quantize(synthetic.bits(x[r0:r0 + rows]))
+    oracle.gemm_mx(qx, sfx, qw[c0:c0 + cols], sfw[c0:c0 + cols], want_bound=False)
+
+
+def cpu_baseline(rows: int, prepared=None):
+    import oracle as _o
+    oracle, synthetic, x, qw, sfw = prepared or _oracle_workload()
+    t = time.perf_counter()
+    _oracle_step(oracle, synthetic, x, qw, sfw, 0, rows)
+    dt = time.perf_counter() - t
+    return {"value": 2.0 * rows * N * K / dt / 1e12, "unit": "TFLOPS", "cores": min(_o.default_threads(), rows),
+            "kind": "oracle", "seconds": dt,
+            "sample": f"{rows} of {M} rows of the ffn_up step (mx-quantize those rows of X, then their full "
+                      f"rows of C against all {N} columns, fp64 exact accumulation); W quantized beforehand"}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    prepared = _oracle_workload()
+    oracle, synthetic, x, qw, sfw = prepared
+    def ref_step(i):
+        r0 = (i * REF_ROWS_PER_STEP) % M
+        c0 = (i * REF_COLS_PER_STEP) % (N - REF_COLS_PER_STEP + 1)
+        _oracle_step(oracle, synthetic, x, qw, sfw, r0, REF_ROWS_PER_STEP, c0, REF_COLS_PER_STEP)
+
+    for i in range(args.warmup):
+        ref_step(i)
+    t = time.perf_counter()
+    for i in range(args.steps):
+        ref_step(args.warmup + i)
+    dt = time.perf_counter() - t
+    value = 2.0 * REF_ROWS_PER_STEP * REF_COLS_PER_STEP * K * args.steps / dt / 1e12
+    sample = (f"each step: a {REF_ROWS_PER_STEP} x {REF_COLS_PER_STEP} block of C of the ffn_up step "
+              f"(mx-quantize those rows of X, exact fp64 dot products over all K = {K})")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "ffn_up 8192x22016x8192 MXFP8 (CPU oracle, sampled rows)",
+                                            "M": M, "N": N, "K": K},
+            "cpu_baseline": {"kind": "oracle", "cores": min(oracle.default_threads(), REF_ROWS_PER_STEP),
+                             "sample": sample, "value": value,
+                             "unit": "TFLOPS"},
+            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
