@@ -180,6 +180,41 @@ fp8mm_status fp8mm_selftest_wait_timeout(uint32_t timeout_us, void* stream);
 /* ABI version of this header: major * 10000 + minor * 100 + patch. */
 int fp8mm_version(void);
 
+
+/* ------------------------------------------------- no-allocation variant */
+
+/* Small-M MXFP8 GEMM (the same arithmetic and kernel as mxfp8_gemm with
+ * m <= 64) for callers that cannot allocate device memory.  The source pages
+ * have no counterpart: this entry point exists for how the library is called,
+ * not for what it computes.
+ *
+ * Who needs it: a caller whose device memory is fully reserved up front by
+ * its own pool (a serving engine that hands nearly all HBM to its KV cache),
+ * a caller on a latency-critical path where cudaMalloc's implicit device
+ * synchronisation is not acceptable, or a plain-C host with no allocator for
+ * the split-K workspace that mxfp8_gemm needs.  Such a caller still passes
+ * its inputs and output; the split-K partial sums and arrival counters live
+ * in a fixed 8 MiB array inside the library (FP8MM_NOALLOC_SCRATCH_BYTES),
+ * which every GPU that loads the library holds until the process exits.
+ *
+ *   a [m, k], sf_a, b [n, k], sf_b, c [m, n] (row stride ldc): as in
+ *   mxfp8_gemm.  Requires 1 <= m <= 64 (else FP8MM_ERR_SHAPE), k % 32 == 0,
+ *   and at most 16384 weight tiles, i.e. n <= 2097152 (else
+ *   FP8MM_ERR_WORKSPACE: the request does not fit the fixed scratch).  The
+ *   stream-K split uses as many CTAs as the scratch holds, up to one per SM.
+ *
+ * Allocates nothing: no cudaMalloc / cudaFree and no allocating library
+ * call.  The first call on each device looks up the scratch array's device
+ * address (cudaGetSymbolAddress, with that device current) and caches it;
+ * make that first call before any stream capture.  Every call clears the
+ * counters it uses (an async memset on `stream`) before its kernel runs.
+ * All calls share the one array, which keeps the last call's contents, so
+ * calls that overlap on the GPU (e.g. on two streams) race: serialise them. */
+#define FP8MM_NOALLOC_SCRATCH_BYTES (8u << 20)
+fp8mm_status mxfp8_gemm_small_m_noalloc(const void* a_e4m3, const uint8_t* sf_a, const void* b_e4m3,
+                                        const uint8_t* sf_b, int64_t m, int64_t n, int64_t k, void* c_bf16,
+                                        int64_t ldc, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

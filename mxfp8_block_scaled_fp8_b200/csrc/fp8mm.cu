@@ -447,3 +447,86 @@ fp8mm_status fp8mm_selftest_wait_timeout(uint32_t timeout_us, void* stream) {
 }
 
 }  // extern "C"
+
+// ====================================================================== no-allocation variant
+// The small-M kernel with its split-K scratch in a fixed array inside the
+// library, for callers that cannot allocate (see fp8mm.h).  Nothing above
+// this point is changed by it.
+namespace fp8mm {
+
+constexpr size_t kNoAllocTicketBytes = size_t(64) << 10;  // one u32 per weight tile: 16384 tiles
+constexpr size_t kNoAllocPartialBytes = size_t(FP8MM_NOALLOC_SCRATCH_BYTES) - kNoAllocTicketBytes;
+
+// Partial sums first, arrival counters in the last 64 KiB.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FP8MM_NOALLOC_SCRATCH_BYTES];
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code may not use the symbol itself as a device pointer).
+static fp8mm_status noalloc_scratch(int dev, unsigned char** out) {
+  static unsigned char* addr[64] = {};
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return cuda_fail(e == cudaSuccess ? cudaErrorInvalidSymbol : e);
+    addr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = addr[dev];
+  return FP8MM_OK;
+}
+
+}  // namespace fp8mm
+
+extern "C" fp8mm_status mxfp8_gemm_small_m_noalloc(const void* a_e4m3, const uint8_t* sf_a, const void* b_e4m3,
+                                                   const uint8_t* sf_b, int64_t m, int64_t n, int64_t k,
+                                                   void* c_bf16, int64_t ldc, void* stream) {
+  fp8mm_status st = check_gemm_common(a_e4m3, b_e4m3, m, n, k, c_bf16, ldc, 32);
+  if (st != FP8MM_OK) return st;
+  if (m > 64) return FP8MM_ERR_SHAPE;
+  if (m == 0 || n == 0) return FP8MM_OK;
+  if (k > 0 && (sf_a == nullptr || sf_b == nullptr)) return FP8MM_ERR_NULL;
+  if (!aligned(sf_a, 16) || !aligned(sf_b, 16)) return FP8MM_ERR_ALIGN;
+  const int64_t n_tiles = cdiv(n, 128);
+  if (static_cast<size_t>(n_tiles) * sizeof(unsigned) > kNoAllocTicketBytes) return FP8MM_ERR_WORKSPACE;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != FP8MM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (k == 0) return zero_output(c_bf16, m, n, ldc, s);
+  unsigned char* scratch = nullptr;
+  if ((st = noalloc_scratch(dev.device, &scratch)) != FP8MM_OK) return st;
+
+  const int nm = small_m_tile(m);
+  DecodeArgs p{};
+  p.m = static_cast<int>(m);
+  p.n = static_cast<int>(n);
+  p.k = static_cast<int>(k);
+  p.num_k = static_cast<int>(cdiv(k, 128));
+  p.n_tiles = static_cast<int>(n_tiles);
+  p.units = static_cast<int64_t>(p.n_tiles) * p.num_k;
+  p.c = static_cast<__nv_bfloat16*>(c_bf16);
+  p.ldc = ldc;
+  p.sfw = sf_b;
+  p.sfx = sf_a;
+  p.n_kc = p.num_k;
+  p.timeout_ns = wait_timeout_ns();
+  // as many CTAs as the partial-sum region holds (2 slots of 128 x nm fp32 each)
+  const int64_t per_cta = 2 * static_cast<int64_t>(nm) * 128 * static_cast<int64_t>(sizeof(float));
+  int64_t g = std::min<int64_t>(dev.sms, static_cast<int64_t>(kNoAllocPartialBytes) / per_cta);
+  g = std::max<int64_t>(1, std::min<int64_t>(g, p.units));
+  p.ctas = static_cast<int>(g);
+  p.partials = reinterpret_cast<float*>(scratch);
+  p.tickets = reinterpret_cast<unsigned*>(scratch + kNoAllocPartialBytes);
+  // the counters must start at zero; a previous call that stopped early may have left some set
+  cudaError_t e = cudaMemsetAsync(p.tickets, 0, static_cast<size_t>(n_tiles) * sizeof(unsigned), s);
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  CUtensorMap tw, tx;
+  if ((st = make_map(&tw, b_e4m3, k, n, 128)) != FP8MM_OK) return st;
+  if ((st = make_map(&tx, a_e4m3, k, m, nm)) != FP8MM_OK) return st;
+  switch (nm) {
+    case 16: return launch_small_m_t<16>(tw, tx, p, s, dev.device);
+    case 32: return launch_small_m_t<32>(tw, tx, p, s, dev.device);
+    case 48: return launch_small_m_t<48>(tw, tx, p, s, dev.device);
+    default: return launch_small_m_t<64>(tw, tx, p, s, dev.device);
+  }
+}

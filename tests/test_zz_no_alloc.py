@@ -1,0 +1,79 @@
+"""The no-allocation small-M GEMM (for callers that cannot allocate device
+memory: its split-K scratch lives in a fixed array inside the library) must
+agree with the regular mxfp8_gemm entry point, which uses a caller-owned
+workspace.  It is called through the C ABI, twice in a row, and checked with
+the same acceptance bar as the other GEMM tests.  Collected last on purpose,
+and independent of every other test."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import mxfp8_block_scaled_fp8_b200 as fp8mm
+from mxfp8_block_scaled_fp8_b200 import fp8mm as binding
+from mxfp8_block_scaled_fp8_b200 import synthetic
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+def _entry():
+    lib = ctypes.CDLL(binding.LIB_PATH)
+    fn = lib.mxfp8_gemm_small_m_noalloc
+    P, I64 = ctypes.c_void_p, ctypes.c_int64
+    fn.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
+    fn.restype = ctypes.c_int
+    return fn
+
+
+def _bound(x_cpu, w_cpu):
+    """Sum_k |a_k b_k| of the dequantized operands, from the CPU oracle."""
+    import oracle
+    qx, sfx = oracle.mx_quantize(synthetic.bits(x_cpu))
+    qw, sfw = oracle.mx_quantize(synthetic.bits(w_cpu))
+    _, bound = oracle.gemm_mx(qx, sfx, qw, sfw)
+    return bound
+
+
+CASES = [  # (m, n, k, label)
+    (1, 6144, 4096, "qkv m=1"),
+    (8, 14336, 4096, "up m=8"),
+    (64, 4096, 14336, "down m=64"),
+    (17, 130, 4128, "ragged"),
+]
+
+
+@pytest.mark.parametrize("m,n,k,label", CASES, ids=[c[3] for c in CASES])
+def test_no_alloc_matches_regular_entry_point(m, n, k, label):
+    gu.require_gpu()
+    fn = _entry()
+    x_cpu = synthetic.random_bf16((m, k), seed=100 + m)
+    w_cpu = synthetic.random_bf16((n, k), seed=200 + n, sigma=0.02)
+    qx, sfx = fp8mm.mxfp8_quantize(x_cpu.cuda())
+    qw, sfw = fp8mm.mxfp8_quantize(w_cpu.cuda())
+    ws = torch.zeros(fp8mm.workspace_bytes(m, n, k), dtype=torch.uint8, device="cuda")
+    c_regular = fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, workspace=ws)
+    torch.cuda.synchronize()
+    bound = _bound(x_cpu, w_cpu)
+    ref = c_regular.float().cpu().numpy().astype(np.float64)
+    stream = torch.cuda.current_stream().cuda_stream
+    outs = []
+    for _ in range(2):                                     # two calls in a row share the scratch
+        c = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device="cuda")
+        st = fn(qx.data_ptr(), sfx.data_ptr(), qw.data_ptr(), sfw.data_ptr(), m, n, k, c.data_ptr(), n, stream)
+        assert st == 0, f"status {st}"
+        torch.cuda.synchronize()
+        gu.check_gemm(c, ref, bound, f"no-alloc vs regular, {label}")
+        outs.append(c)
+    assert torch.equal(outs[0], outs[1])
+    assert fp8mm.last_device_error() == 0
+
+
+def test_no_alloc_rejects_what_does_not_fit():
+    gu.require_gpu()
+    fn = _entry()
+    dummy = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+    p = dummy.data_ptr()
+    assert fn(p, p, p, p, 65, 128, 128, p, 128, None) == 2              # m > 64
+    assert fn(p, p, p, p, 8, 128 * 16385, 128, p, 128 * 16385, None) == 6   # more tiles than counters
