@@ -154,96 +154,130 @@ def _dist():
 
 # ---------------------------------------------------------------- GPU timing utilities
 
-def _timed(fn, reps, warmup, flush=None, stream=None):
-    """Median device time (ms) of fn over reps, CUDA events on the launching
-    stream, L2 flushed (outside the events) before each rep when given."""
+def _graph_time(calls, reps: int = 10) -> float:
+    """Device time (ms) per call: `calls` (one zero-argument function per
+    call, each touching its own copy of the large operand so that together
+    they exceed L2) are captured once into a CUDA graph and replayed `reps`
+    times between two CUDA events.  This times the kernels back to back, as a
+    serving engine replays them, without host launch latency."""
     import torch
-    s = stream or torch.cuda.current_stream()
-    for _ in range(warmup):
-        fn()
-    times = []
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for f in calls:                      # first calls: per-device setup happens here
+            f()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for f in calls:
+            f()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
     for _ in range(reps):
-        if flush is not None:
-            flush()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(s)
-        fn()
-        b.record(s)
-        b.synchronize()
-        times.append(a.elapsed_time(b))
-    return statistics.median(times), min(times)
+        g.replay()
+    b.record()
+    b.synchronize()
+    ms = a.elapsed_time(b) / (reps * len(calls))
+    del g
+    return ms
 
 
-def _rows_measurements(fp8mm, synthetic, peaks, reps=20):
-    """Per-row measurements of the other hot-path steps (each its own unit)."""
+def _copies(nbytes: int, min_total: int = 320 << 20) -> int:
+    return max(2, -(-min_total // max(nbytes, 1)))
+
+
+def _rows_measurements(fp8mm, synthetic, peaks, only=None):
+    """Per-row measurements of the other hot-path steps (each its own unit),
+    timed by CUDA-graph replay over rotated operand copies (> L2 in total)."""
+    import re
     import torch
     dev = torch.device("cuda")
-    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    flush = lambda: flush_buf.zero_()
     out = {}
     hbm = peaks["hbm_gbs"]
     fp8_peak = 2.0 * peaks["bf16_tflops"]
+    want = (lambda name: re.search(only, name) is not None) if only else (lambda name: True)
 
-    # per-row quantizer and rowwise GEMM on the attention-like workload
-    a, bt = synthetic.attn()
-    a, bt = a.to(dev), bt.to(dev)
-    qa = torch.empty(a.shape, dtype=torch.uint8, device=dev)
-    sa = torch.empty(a.shape[0], dtype=torch.float32, device=dev)
-    t, _ = _timed(lambda: fp8mm.fp8_quantize_rowwise(a, qa, sa), reps, 3, flush)
-    R, Kq = a.shape
-    gbs = (3.0 * R * Kq + 4 * R) / (t * 1e-3) / 1e9
-    out["quantize_rowwise_8192x8192"] = {"ms": t, "GB/s": gbs, "frac_hbm": gbs / hbm}
-    qb, sb = fp8mm.fp8_quantize_rowwise(bt)
-    c = torch.empty((a.shape[0], bt.shape[0]), dtype=torch.bfloat16, device=dev)
-    t, _ = _timed(lambda: fp8mm.fp8_gemm(qa, qb, sa, sb, c), reps, 3, flush)
-    tf = 2.0 * 8192 * 2048 * 8192 / (t * 1e-3) / 1e12
-    out["fp8_gemm_8192x2048x8192"] = {"ms": t, "TFLOPS": tf, "frac_fp8_peak": tf / fp8_peak}
-    del a, bt, qa, qb, c
+    if want("quantize_rowwise_8192x8192") or want("fp8_gemm_8192x2048x8192"):
+        a, bt = synthetic.attn()
+        a, bt = a.to(dev), bt.to(dev)
+        R, Kq = a.shape
+        if want("quantize_rowwise_8192x8192"):
+            xs = [a] + [a.clone() for _ in range(_copies(a.numel() * 2) - 1)]
+            qa = torch.empty(a.shape, dtype=torch.uint8, device=dev)
+            sa = torch.empty(R, dtype=torch.float32, device=dev)
+            t = _graph_time([lambda x=x: fp8mm.fp8_quantize_rowwise(x, qa, sa) for x in xs])
+            gbs = (3.0 * R * Kq + 4 * R) / (t * 1e-3) / 1e9
+            out["quantize_rowwise_8192x8192"] = {"ms": t, "GB/s": gbs, "frac_hbm": gbs / hbm}
+            del xs
+        if want("fp8_gemm_8192x2048x8192"):
+            qa, sa = fp8mm.fp8_quantize_rowwise(a)
+            qb, sb = fp8mm.fp8_quantize_rowwise(bt)
+            c = torch.empty((R, bt.shape[0]), dtype=torch.bfloat16, device=dev)
+            t = _graph_time([lambda: fp8mm.fp8_gemm(qa, qb, sa, sb, c)] * 4)
+            tf = 2.0 * 8192 * 2048 * 8192 / (t * 1e-3) / 1e12
+            out["fp8_gemm_8192x2048x8192"] = {"ms": t, "TFLOPS": tf, "frac_fp8_peak": tf / fp8_peak}
+        del a, bt
 
-    # MX Q.K^T shape (64 output tiles: fewer than the 148 SMs)
-    a, bt = synthetic.qk()
-    qa, sfa = fp8mm.mxfp8_quantize(a.to(dev))
-    qb, sfb = fp8mm.mxfp8_quantize(bt.to(dev))
-    c = torch.empty((2048, 1024), dtype=torch.bfloat16, device=dev)
-    t, _ = _timed(lambda: fp8mm.mxfp8_gemm(qa, sfa, qb, sfb, c), reps, 3, flush)
-    tf = 2.0 * 2048 * 1024 * 4096 / (t * 1e-3) / 1e12
-    out["mxfp8_gemm_2048x1024x4096"] = {"ms": t, "TFLOPS": tf, "frac_fp8_peak": tf / fp8_peak}
+    if want("mxfp8_gemm_2048x1024x4096"):
+        # Q.K^T shape: 64 output tiles, fewer than the 148 SMs
+        a, bt = synthetic.qk()
+        qa, sfa = fp8mm.mxfp8_quantize(a.to(dev))
+        qb, sfb = fp8mm.mxfp8_quantize(bt.to(dev))
+        c = torch.empty((2048, 1024), dtype=torch.bfloat16, device=dev)
+        t = _graph_time([lambda: fp8mm.mxfp8_gemm(qa, sfa, qb, sfb, c)] * 8)
+        tf = 2.0 * 2048 * 1024 * 4096 / (t * 1e-3) / 1e12
+        out["mxfp8_gemm_2048x1024x4096"] = {"ms": t, "TFLOPS": tf, "frac_fp8_peak": tf / fp8_peak}
 
-    # MX quantizer on the FFN weight (done once at load) -- measured standalone
-    _, w = synthetic.ffn_up()
-    w = w.to(dev)
-    qw = torch.empty(w.shape, dtype=torch.uint8, device=dev)
-    sfw = torch.empty(fp8mm.sf_bytes(*w.shape), dtype=torch.uint8, device=dev)
-    t, _ = _timed(lambda: fp8mm.mxfp8_quantize(w, qw, sfw), reps, 3, flush)
-    R, Kq = w.shape
-    gbs = (3.0 * R * Kq + R * Kq / 32) / (t * 1e-3) / 1e9
-    out["mxfp8_quantize_22016x8192"] = {"ms": t, "GB/s": gbs, "frac_hbm": gbs / hbm}
-    del w, qw, sfw
+    if want("mxfp8_quantize_22016x8192"):
+        # MX quantizer on the FFN weight (done once at load), standalone
+        _, w = synthetic.ffn_up()
+        w = w.to(dev)
+        qw = torch.empty(w.shape, dtype=torch.uint8, device=dev)
+        sfw = torch.empty(fp8mm.sf_bytes(*w.shape), dtype=torch.uint8, device=dev)
+        t = _graph_time([lambda: fp8mm.mxfp8_quantize(w, qw, sfw)] * 2)
+        R, Kq = w.shape
+        gbs = (3.0 * R * Kq + R * Kq / 32) / (t * 1e-3) / 1e9
+        out["mxfp8_quantize_22016x8192"] = {"ms": t, "GB/s": gbs, "frac_hbm": gbs / hbm}
+        del w, qw, sfw
 
     # decode sweep: quantize X per call + small-M GEMM against a resident weight
     ws_, xs = synthetic.decode()
     sweep = {}
     for name, w in ws_.items():
         n, k = synthetic.DECODE_SHAPES[name]
-        qw, sfw = fp8mm.mxfp8_quantize(w.to(dev))
+        if not any(want(f"{name}_{n}x{k}_m{m}") for m in synthetic.DECODE_M):
+            continue
+        qw0, sfw0 = fp8mm.mxfp8_quantize(w.to(dev))
+        copies = _copies(qw0.numel())
+        wq = [(qw0, sfw0)] + [(qw0.clone(), sfw0.clone()) for _ in range(copies - 1)]
         for m in synthetic.DECODE_M:
+            key = f"{name}_{n}x{k}_m{m}"
+            if not want(key):
+                continue
             x = xs[k][:m].contiguous().to(dev)
             qx = torch.empty((m, k), dtype=torch.uint8, device=dev)
             sfx = torch.empty(fp8mm.sf_bytes(m, k), dtype=torch.uint8, device=dev)
             c = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
             wsp = torch.zeros(fp8mm.workspace_bytes(m, n, k), dtype=torch.uint8, device=dev)
 
-            def call():
+            def call(qw, sfw):
                 fp8mm.mxfp8_quantize(x, qx, sfx)
                 fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c, workspace=wsp)
-            t, _ = _timed(call, reps, 3, flush)
-            tg, _ = _timed(lambda: fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c, workspace=wsp), reps, 3, flush)
+            t = _graph_time([lambda qw=qw, sfw=sfw: call(qw, sfw) for qw, sfw in wq])
+            tg = _graph_time([lambda qw=qw, sfw=sfw: fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c, workspace=wsp)
+                              for qw, sfw in wq])
             e2e_bytes = n * k + n * k / 32 + 2 * m * k + 2 * m * n
             gemm_bytes = n * k + n * k / 32 + m * k + 128 * k / 32 + 2 * m * n
-            sweep[f"{name}_{n}x{k}_m{m}"] = {
-                "ms": t, "GB/s": e2e_bytes / (t * 1e-3) / 1e9, "frac_hbm": e2e_bytes / (t * 1e-3) / 1e9 / hbm,
-                "gemm_ms": tg, "gemm_GB/s": gemm_bytes / (tg * 1e-3) / 1e9}
-    out["decode"] = sweep
+            sweep[key] = {"ms": t, "GB/s": e2e_bytes / (t * 1e-3) / 1e9, "frac_hbm": e2e_bytes / (t * 1e-3) / 1e9 / hbm,
+                          "gemm_ms": tg, "gemm_GB/s": gemm_bytes / (tg * 1e-3) / 1e9,
+                          "gemm_frac_hbm": gemm_bytes / (tg * 1e-3) / 1e9 / hbm}
+        del wq
+    if sweep:
+        out["decode"] = sweep
+    out["timing"] = "CUDA-graph replay, operands rotated over copies totalling > 320 MiB (no L2 reuse)"
     return out
 
 
@@ -334,7 +368,7 @@ def run_ours(args):
 
     rows = None
     if rank == 0 and not args.no_rows:
-        rows = _rows_measurements(fp8mm, synthetic, peaks)
+        rows = _rows_measurements(fp8mm, synthetic, peaks, args.only)
 
     fp8_peak = 2.0 * peaks["bf16_tflops"]
     achieved = FLOPS_PER_STEP / (g_ms * 1e-3) / 1e12
@@ -442,9 +476,17 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--only", default=None, help="regex: measure only the matching per-row cases")
+    ap.add_argument("--rows-only", action="store_true", help="skip the headline step (profiling of single rows)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.rows_only:
+        import torch
+        import mxfp8_block_scaled_fp8_b200 as fp8mm
+        from mxfp8_block_scaled_fp8_b200 import synthetic
+        torch.cuda.set_device(0)
+        print(json.dumps({"rows": _rows_measurements(fp8mm, synthetic, _peaks(), args.only)}), flush=True)
     else:
         run_ours(args)
 

@@ -68,9 +68,13 @@ typedef struct fp8mm_opts {
    * the GPU.  NULL disables split-K. */
   void* workspace;
   size_t workspace_bytes;
-  /* Kernel choice: FP8MM_KERNEL_AUTO, FP8MM_KERNEL_TILED (persistent 128x256
-   * tiles) or FP8MM_KERNEL_SMALL_M (weights on the MMA M side, tokens on N;
-   * mxfp8_gemm only, m <= 64). */
+  /* Kernel choice: FP8MM_KERNEL_AUTO (small-M kernel for mxfp8_gemm with
+   * m <= 64, paired-SM tiles for m >= 256, single-SM tiles otherwise),
+   * FP8MM_KERNEL_TILED (tiled, pair or single chosen by size),
+   * FP8MM_KERNEL_SMALL_M (weights on the MMA M side, tokens on N; mxfp8_gemm
+   * only, m <= 64), FP8MM_KERNEL_TILED_1SM (persistent 128x256 tiles, one CTA
+   * per SM) or FP8MM_KERNEL_TILED_2SM (256x256 tiles on 2-CTA clusters with
+   * cta_group::2 MMAs; each CTA loads its own halves of A and B). */
   int32_t kernel;
   /* Number of CTAs for the small-M kernel's stream-K split (0 = one per SM). */
   int32_t small_m_ctas;
@@ -79,6 +83,8 @@ typedef struct fp8mm_opts {
 #define FP8MM_KERNEL_AUTO 0
 #define FP8MM_KERNEL_TILED 1
 #define FP8MM_KERNEL_SMALL_M 2
+#define FP8MM_KERNEL_TILED_1SM 3
+#define FP8MM_KERNEL_TILED_2SM 4
 
 /* ---------------------------------------------------------------- mode 1 */
 

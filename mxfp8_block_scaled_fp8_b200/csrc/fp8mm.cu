@@ -15,6 +15,7 @@
 
 #include "decode.cuh"
 #include "gemm.cuh"
+#include "gemm2.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 
@@ -111,6 +112,24 @@ static fp8mm_status make_map(CUtensorMap* map, const void* base, int64_t k, int6
   return FP8MM_OK;
 }
 
+// 3-D map over a library scale buffer viewed as uint32 [n_rt][n_kc][128]
+// (one 512-byte chunk per 128-row tile and 4-block group); box = box_rt chunks
+// of consecutive row tiles at one K group; zero fill past the last row tile.
+static fp8mm_status make_sf_map(CUtensorMap* map, const void* sf, int64_t k, int64_t rows, int box_rt) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
+  const int64_t n_kc = (k + 127) / 128, n_rt = (rows + 127) / 128;
+  cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(n_kc), static_cast<cuuint64_t>(n_rt)};
+  cuuint64_t strides[2] = {512u, static_cast<cuuint64_t>(n_kc) * 512u};
+  cuuint32_t box[3] = {128u, 1u, static_cast<cuuint32_t>(box_rt)};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(sf), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return FP8MM_OK;
+}
+
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -173,6 +192,99 @@ static fp8mm_status launch_tiled(bool mx, const void* a, const void* b, const ui
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), G1::kSmemBytes, dev.device)) != FP8MM_OK) return st;
     kern<<<grid, kGemmThreads, G1::kSmemBytes, stream>>>(ta, tb, p);
   }
+  return launched();
+}
+
+using P1 = PairCfg<false, 6, 2>;
+using P2 = PairCfg<true, 6, 1>;
+
+// Largest number of co-resident 2-CTA clusters of a pair kernel (cached).
+static fp8mm_status max_pairs(const void* kern, int smem, const DeviceInfo& dev, int* out) {
+  static std::set<std::pair<const void*, int>> done;
+  static int cached[2][64];
+  const int which = (kern == reinterpret_cast<const void*>(gemm_pair_kernel<true, 6, 1>)) ? 1 : 0;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (done.count({kern, dev.device})) {
+      *out = cached[which][dev.device];
+      return FP8MM_OK;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * (dev.sms / 2), 1, 1);
+  cfg.blockDim = dim3(which ? P2::kThreads : P1::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (n <= 0) n = 1;
+  std::lock_guard<std::mutex> lock(g_mu);
+  cached[which][dev.device] = n;
+  done.insert({kern, dev.device});
+  *out = n;
+  return FP8MM_OK;
+}
+
+static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uint8_t* sfa, const uint8_t* sfb,
+                                int64_t m, int64_t n, int64_t k, const float* sa, const float* sb, void* c,
+                                int64_t ldc, cudaStream_t stream, const DeviceInfo& dev) {
+  CUtensorMap ta, tb, tsa, tsb;
+  fp8mm_status st = make_map(&ta, a, k, m, 128);
+  if (st != FP8MM_OK) return st;
+  if ((st = make_map(&tb, b, k, n, 128)) != FP8MM_OK) return st;
+  if (mx) {
+    if ((st = make_sf_map(&tsa, sfa, k, m, 1)) != FP8MM_OK) return st;
+    if ((st = make_sf_map(&tsb, sfb, k, n, 2)) != FP8MM_OK) return st;
+  } else {
+    tsa = ta;  // unused in per-token mode
+    tsb = tb;
+  }
+  GemmArgs p{};
+  p.m = static_cast<int>(m);
+  p.n = static_cast<int>(n);
+  p.k = static_cast<int>(k);
+  p.num_k = static_cast<int>(cdiv(k, kBK));
+  p.tiles_m = static_cast<int>(cdiv(m, 256));
+  p.tiles_n = static_cast<int>(cdiv(n, 256));
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.c = static_cast<__nv_bfloat16*>(c);
+  p.ldc = ldc;
+  p.sa = sa;
+  p.sb = sb;
+  p.sfa = sfa;
+  p.sfb = sfb;
+  p.n_kc = static_cast<int>(cdiv(k, 128));
+  p.sfb_row_tiles = static_cast<int>(cdiv(n, 128));
+  p.timeout_ns = wait_timeout_ns();
+  const void* kern = mx ? reinterpret_cast<const void*>(gemm_pair_kernel<true, 6, 1>)
+                        : reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2>);
+  const int smem = mx ? P2::kSmemBytes : P1::kSmemBytes;
+  if ((st = ensure_smem(kern, smem, dev.device)) != FP8MM_OK) return st;
+  int pairs = 0;
+  if ((st = max_pairs(kern, smem, dev, &pairs)) != FP8MM_OK) return st;
+  pairs = std::min(pairs, p.num_tiles);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(mx ? P2::kThreads : P1::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = mx ? cudaLaunchKernelEx(&cfg, gemm_pair_kernel<true, 6, 1>, ta, tb, tsa, tsb, p)
+                     : cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false, 6, 2>, ta, tb, tsa, tsb, p);
+  if (e != cudaSuccess) return cuda_fail(e);
   return launched();
 }
 
@@ -360,13 +472,11 @@ fp8mm_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
   fp8mm_status st = current_device(&dev);
   if (st != FP8MM_OK) return st;
   const int64_t n_kc = cdiv(k, 128);
-  const int64_t n_groups = cdiv(rows, 128) * 128 * n_kc;
-  const int64_t groups_per_cta_step = (kQ2Threads / 32) * 2;
-  const int64_t want = cdiv(n_groups, groups_per_cta_step * kQ2Unroll);
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(dev.sms) * 8)));
+  const int64_t rows_pad = cdiv(rows, 128) * 128;
+  const int grid = static_cast<int>(std::min<int64_t>(rows_pad, static_cast<int64_t>(dev.sms) * 8));
   quant_mx_kernel<<<grid, kQ2Threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x_bf16), rows, k, ld_x, static_cast<uint8_t*>(q_e4m3), ld_q, sf, n_kc,
-      n_groups);
+      static_cast<const __nv_bfloat16*>(x_bf16), rows, k, ld_x, static_cast<uint8_t*>(q_e4m3), ld_q, sf,
+      static_cast<int>(n_kc), rows_pad);
   return launched();
 }
 
@@ -392,11 +502,16 @@ fp8mm_status fp8_gemm(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t
   if (st != FP8MM_OK || m == 0 || n == 0) return st;
   if (k > 0 && (scale_a == nullptr || scale_b == nullptr)) return FP8MM_ERR_NULL;
   if (!aligned(scale_a, 4) || !aligned(scale_b, 4)) return FP8MM_ERR_ALIGN;
-  if (opt != nullptr && opt->kernel == FP8MM_KERNEL_SMALL_M) return FP8MM_ERR_SHAPE;
+  if (opt != nullptr && (opt->kernel == FP8MM_KERNEL_SMALL_M || opt->kernel < FP8MM_KERNEL_AUTO ||
+                         opt->kernel > FP8MM_KERNEL_TILED_2SM))
+    return FP8MM_ERR_SHAPE;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != FP8MM_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (k == 0) return zero_output(c_bf16, m, n, ldc, s);
+  const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
+  const bool pair = (kind == FP8MM_KERNEL_TILED_2SM) || (kind != FP8MM_KERNEL_TILED_1SM && m >= 256);
+  if (pair) return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev);
   return launch_tiled(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev);
 }
 
@@ -408,13 +523,15 @@ fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e
   if (!aligned(sf_a, 16) || !aligned(sf_b, 16)) return FP8MM_ERR_ALIGN;
   const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
   if (kind == FP8MM_KERNEL_SMALL_M && m > 64) return FP8MM_ERR_SHAPE;
-  if (kind < FP8MM_KERNEL_AUTO || kind > FP8MM_KERNEL_SMALL_M) return FP8MM_ERR_SHAPE;
+  if (kind < FP8MM_KERNEL_AUTO || kind > FP8MM_KERNEL_TILED_2SM) return FP8MM_ERR_SHAPE;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != FP8MM_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (k == 0) return zero_output(c_bf16, m, n, ldc, s);
   const bool small = (kind == FP8MM_KERNEL_SMALL_M) || (kind == FP8MM_KERNEL_AUTO && m <= 64);
   if (small) return launch_small_m(a_e4m3, sf_a, b_e4m3, sf_b, m, n, k, c_bf16, ldc, opt, s, dev);
+  const bool pair = (kind == FP8MM_KERNEL_TILED_2SM) || (kind != FP8MM_KERNEL_TILED_1SM && m >= 256);
+  if (pair) return launch_pair(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev);
   return launch_tiled(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev);
 }
 

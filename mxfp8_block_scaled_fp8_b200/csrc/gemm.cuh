@@ -15,9 +15,9 @@
 //               the 512-byte scale chunks, into a kStages-deep ring.
 //   warp 1      allocates TMEM; one lane issues tcgen05.mma (and tcgen05.cp of
 //               the scale chunks) per 128-byte K slab, commits to free the slab.
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (each warp owns
-//               the 32 TMEM lanes of its sub-partition), scaling, bf16 RNE,
-//               stores.
+//   warps 2..9  epilogue: each drains half a tile row-block of the fp32
+//               accumulator into registers (tcgen05.ld, one wait), frees the
+//               accumulator, then scales, converts to bf16 RNE and stores.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -30,7 +30,7 @@ namespace fp8mm {
 constexpr int kBM = 128;            // tile rows (A / M side of the MMA)
 constexpr int kBK = 128;            // K elements (= bytes) per pipeline slab
 constexpr int kMmaK = 32;           // K per tcgen05.mma for 8-bit operands
-constexpr int kGemmThreads = 192;   // 6 warps
+constexpr int kGemmThreads = 320;   // 10 warps: producer, MMA, 8 epilogue
 constexpr int kGroupM = 16;
 
 struct GemmArgs {
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < kAccStages; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], 8);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -230,7 +230,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------ epilogue
-    const int sp = warp & 3;  // TMEM sub-partition this warp can read
+    // Eight warps: warp w reads TMEM sub-partition (w % 4), i.e. tile rows
+    // 32*(w%4) .. +31, and one half of the tile's columns.  Each thread pulls
+    // its 128 accumulator values into registers with four loads and a single
+    // wait, then releases the accumulator at once, so the next tile's MMAs
+    // overlap the scaling, conversion and stores below.
+    const int sp = warp & 3;
+    const int col_half = (warp - 2) >> 2;
+    constexpr int kHalf = kBN / 2;
+    static_assert(kHalf == 128, "epilogue assumes 256-column tiles");
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
@@ -238,28 +246,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tile_coords(t, p, mb, nb);
       if (!mbar_wait(&acc_full[acc], acc_phase, p.timeout_ns, abort_flag, kSiteEpiAccFull)) break;
       tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) +
+                             static_cast<uint32_t>(acc * kBN + col_half * kHalf);
+      uint32_t r[4][32];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_ld_32x32b_x32(t_row + ch * 32, r[ch]);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) asm volatile("" : FP8MM_RW32(r[ch]));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (++acc == kAccStages) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+
       const int row = mb * kBM + sp * 32 + lane;
       float s_row = 1.f;
       if constexpr (!kMX) s_row = (row < p.m) ? __ldg(p.sa + row) : 0.f;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(acc * kBN);
-#pragma unroll 1
-      for (int ch = 0; ch < kBN / 32; ++ch) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + ch * 32, r);
-        tmem_ld_wait_32(r);
-        if (ch == kBN / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        }
-        const int col0 = nb * kBN + ch * 32;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        const int col0 = nb * kBN + col_half * kHalf + ch * 32;
         float sbv = 1.f;
         if constexpr (!kMX) sbv = (col0 + lane < p.n) ? __ldg(p.sb + col0 + lane) : 0.f;
         uint32_t packed[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          float v0 = __uint_as_float(r[2 * j]);
-          float v1 = __uint_as_float(r[2 * j + 1]);
+          float v0 = __uint_as_float(r[ch][2 * j]);
+          float v1 = __uint_as_float(r[ch][2 * j + 1]);
           if constexpr (!kMX) {
             v0 = v0 * s_row * __shfl_sync(0xFFFFFFFFu, sbv, 2 * j);
             v1 = v1 * s_row * __shfl_sync(0xFFFFFFFFu, sbv, 2 * j + 1);
@@ -284,10 +299,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
-      }
-      if (++acc == kAccStages) {
-        acc = 0;
-        acc_phase ^= 1u;
       }
     }
   }

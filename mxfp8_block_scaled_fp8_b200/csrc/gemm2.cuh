@@ -1,0 +1,305 @@
+// gemm2.cuh -- paired-SM tcgen05 GEMM (cta_group::2) for both scale modes.
+//
+// Same arithmetic as gemm.cuh (page "从 DeepGEMM 到 vLLM", listing 1 for the
+// per-token mode; page "[sglang] FlashInfer v0.6.7 MXFP8 Gemm 통합", section 2
+// for the block-scaled mode), computed by 2-CTA clusters on 256 x 256 output
+// tiles.  Each CTA of a pair loads its own 128-row half of the A tile and its
+// own 128-row half of the B tile; nothing is multicast.  Those loads complete
+// on the rank-0 CTA's barrier, whose one thread issues the cta_group::2 MMAs
+// (M = 256, N = 256, K = 32) that read A and B from both CTAs' shared memory
+// and accumulate 128 rows in each CTA's TMEM.  Per 128-byte K slab a CTA moves
+// 32 KiB into shared memory for 128x256x128 MACs, two thirds of what the
+// single-CTA 128x256 tile needs.
+//
+// Block scales (mode 2): each CTA loads its A scale chunk and both B scale
+// chunks (every CTA needs all 256 B rows' scales in its own TMEM) with the
+// same pair-completed TMA loads; the MMA thread copies them into the stage's
+// TMEM columns with tcgen05.cp.cta_group::2 right before that stage's MMAs.
+// Moving the copies to other warps (tcgen05.st from four scale warps, or the
+// copies issued by a second thread) measured no faster, and cluster-scope
+// release arrivals from those warps made the kernel ~45 % slower.
+//
+// Warp roles per CTA: warp 0 TMA producer; warp 1 TMEM owner and, on rank 0,
+// MMA issuer; warps 2..17 epilogue (four per TMEM sub-partition, 64
+// accumulator columns each, drained into registers with one wait so the
+// accumulator is free again at once).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace fp8mm {
+
+constexpr int kPairGroupM = 8;     // 256-row tiles per raster group
+
+template <bool kMX, int kStages, int kAccStages>
+struct PairCfg {
+  // Warps: producer, MMA, 16 epilogue warps.
+  static constexpr int kEpiWarp0 = 2;
+  static constexpr int kThreads = (kEpiWarp0 + 16) * 32;
+  static constexpr int kABytes = 128 * kBK;          // this CTA's half of A
+  static constexpr int kBBytes = 128 * kBK;          // this CTA's half of B
+  static constexpr int kSfaBytes = kMX ? 512 : 0;    // this CTA's 128 A rows x 4 blocks
+  static constexpr int kSfbBytes = kMX ? 1024 : 0;   // all 256 B rows x 4 blocks
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + kStages * kABytes;
+  static constexpr int kOffSfa = kOffB + kStages * kBBytes;
+  static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
+  static constexpr int kOffBar = kOffSfb + kStages * kSfbBytes;
+  // full, empty per stage; acc_full, acc_empty per accumulator; drain
+  static constexpr int kNumBars = 2 * kStages + 2 * kAccStages + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  // bytes of both CTAs' loads, all completing on the leader's barrier
+  static constexpr uint32_t kTxPair = 2u * (kABytes + kBBytes + kSfaBytes + kSfbBytes);
+  static constexpr int kSfColsPerStage = 12;                       // A: 4 columns, B: 8 columns
+  static constexpr int kSfCol0 = kAccStages * 256;
+  static constexpr int kColsUsed = kSfCol0 + (kMX ? kStages * kSfColsPerStage : 0);
+  static constexpr int kTmemCols = kColsUsed <= 256 ? 256 : 512;
+  static_assert(kColsUsed <= 512, "TMEM budget");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ void pair_tile_coords(int t, const GemmArgs& p, int& mb, int& nb) {
+  const int per_group = kPairGroupM * p.tiles_n;
+  const int g = t / per_group;
+  const int first_m = g * kPairGroupM;
+  const int gm = min(p.tiles_m - first_m, kPairGroupM);
+  const int r = t - g * per_group;
+  mb = first_m + r % gm;
+  nb = r / gm;
+}
+
+// GemmArgs fields as in gemm.cuh, with tiles_m = ceil(m/256), tiles_n =
+// ceil(n/256).  tmSFA / tmSFB: 3-D maps over the scale layout viewed as
+// uint32 [n_rt][n_kc][128] (unused in per-token mode).
+template <bool kMX, int kStages, int kAccStages>
+__global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+                     const GemmArgs p) {
+  using Cfg = PairCfg<kMX, kStages, kAccStages>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + kAccStages;
+  uint64_t* drain = acc_empty + kAccStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int pair = static_cast<int>(cluster_id_x());
+  const int npairs = static_cast<int>(num_clusters_x());
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < kAccStages; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 32);  // 16 epilogue warps in each CTA of the pair
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    if constexpr (kMX) {
+      prefetch_tmap(&tmSFA);
+      prefetch_tmap(&tmSFB);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < p.num_tiles; t += npairs) {
+        int mb, nb;
+        pair_tile_coords(t, p, mb, nb);
+        for (int kb = 0; kb < p.num_k; ++kb) {
+          if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[stage], Cfg::kTxPair);
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          tma_load_2d_pair(smem + Cfg::kOffA + stage * Cfg::kABytes, &tmA, fb, kb * kBK, mb * 256 + rank * 128);
+          tma_load_2d_pair(smem + Cfg::kOffB + stage * Cfg::kBBytes, &tmB, fb, kb * kBK, nb * 256 + rank * 128);
+          if constexpr (kMX) {
+            tma_load_3d_pair(smem + Cfg::kOffSfa + stage * Cfg::kSfaBytes, &tmSFA, fb, 0, kb, mb * 2 + rank);
+            tma_load_3d_pair(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes, &tmSFB, fb, 0, kb, nb * 2);
+          }
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Every copy of both CTAs completes on the leader's barriers: the leader
+      // waits for the last phase issued on each stage before the pair may exit.
+      if (leader)
+        for (int s = 0; s < kStages; ++s)
+          if (issued_mask & (1u << s))
+            mbar_wait_cluster(&full[s], (issued_parity >> s) & 1u, p.timeout_ns, nullptr, kSiteProducerDrain);
+      if (!leader && !ok) {
+        // A/B loads of this CTA that the leader never waited for may still be
+        // in flight; give them time to land before the final cluster barrier.
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000ull) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer (rank 0 only)
+    if (leader && lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < p.num_tiles; t += npairs) {
+        if (!mbar_wait_cluster(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, kSiteMmaAccEmpty)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+        for (int kb = 0; kb < p.num_k; ++kb) {
+          if (!mbar_wait_cluster(&full[stage], phase, p.timeout_ns, abort_flag, kSiteMmaFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffA + stage * Cfg::kABytes));
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffB + stage * Cfg::kBBytes));
+          if constexpr (kMX) {
+            const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(Cfg::kSfCol0 + stage * Cfg::kSfColsPerStage);
+            tmem_cp_32x128b_warpx4_pair(sfa_t, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfa + stage * Cfg::kSfaBytes)));
+            tmem_cp_32x128b_warpx4_pair(sfa_t + 4u,
+                                        sf_chunk_desc(smem_u32(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes)));
+            tmem_cp_32x128b_warpx4_pair(sfa_t + 8u,
+                                        sf_chunk_desc(smem_u32(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes + 512)));
+#pragma unroll
+            for (int kk = 0; kk < kBK / kMmaK; ++kk)
+              mma_mxf8f6f4_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8f6f4(256, 256, kk, kk), sfa_t,
+                                sfa_t + 4u, (kb | kk) != 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kBK / kMmaK; ++kk)
+              mma_f8f6f4_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_f8f6f4(256, 256), (kb | kk) != 0);
+          }
+          tc_commit_pair_mc(&empty[stage], 0x3);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&acc_full[acc], 0x3);
+        if (++acc == kAccStages) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      tc_commit_pair_mc(drain, 0x1);
+      mbar_wait(drain, 0, p.timeout_ns, nullptr, kSiteDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------ epilogue (both CTAs)
+    const int sp = warp & 3;
+    const int quarter = (warp - Cfg::kEpiWarp0) >> 2;  // 64-column slice of the 256-column tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < p.num_tiles; t += npairs) {
+      int mb, nb;
+      pair_tile_coords(t, p, mb, nb);
+      if (!mbar_wait_cluster(&acc_full[acc], acc_phase, p.timeout_ns, abort_flag, kSiteEpiAccFull)) break;
+      tc_fence_after();
+      const uint32_t t_row =
+          tmem_base + (static_cast<uint32_t>(sp * 32) << 16) + static_cast<uint32_t>(acc * 256 + quarter * 64);
+      uint32_t r[2][32];
+      tmem_ld_32x32b_x32(t_row, r[0]);
+      tmem_ld_32x32b_x32(t_row + 32, r[1]);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      asm volatile("" : FP8MM_RW32(r[0]));
+      asm volatile("" : FP8MM_RW32(r[1]));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
+      if (++acc == kAccStages) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+
+      const int row = mb * 256 + static_cast<int>(rank) * 128 + sp * 32 + lane;
+      float s_row = 1.f;
+      if constexpr (!kMX) s_row = (row < p.m) ? __ldg(p.sa + row) : 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        const int col0 = nb * 256 + quarter * 64 + ch * 32;
+        float sbv = 1.f;
+        if constexpr (!kMX) sbv = (col0 + lane < p.n) ? __ldg(p.sb + col0 + lane) : 0.f;
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float v0 = __uint_as_float(r[ch][2 * j]);
+          float v1 = __uint_as_float(r[ch][2 * j + 1]);
+          if constexpr (!kMX) {
+            v0 = v0 * s_row * __shfl_sync(0xFFFFFFFFu, sbv, 2 * j);
+            v1 = v1 * s_row * __shfl_sync(0xFFFFFFFFu, sbv, 2 * j + 1);
+          }
+          __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+          packed[j] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        if (row < p.m && col0 < p.n) {
+          __nv_bfloat16* dst = p.c + static_cast<int64_t>(row) * p.ldc + col0;
+          if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              *reinterpret_cast<uint4*>(dst + q4 * 8) =
+                  make_uint4(packed[4 * q4], packed[4 * q4 + 1], packed[4 * q4 + 2], packed[4 * q4 + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (col0 + j < p.n) {
+                const uint32_t w = packed[j >> 1];
+                *reinterpret_cast<uint16_t*>(dst + j) = static_cast<uint16_t>((j & 1) ? (w >> 16) : (w & 0xFFFFu));
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still signal or read it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace fp8mm

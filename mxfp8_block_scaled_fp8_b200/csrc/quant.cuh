@@ -165,65 +165,65 @@ __device__ __forceinline__ float mx_inv_scale(int e) {
   return (e < 254) ? __uint_as_float(static_cast<uint32_t>(254 - e) << 23) : __uint_as_float(0x00400000u);
 }
 
-constexpr int kQ2Threads = 256;
-constexpr int kQ2Unroll = 4;
+constexpr int kQ2Threads = 256;   // 8 warps = 16 groups of 128 elements per pass
+constexpr int kQ2Passes = 8;      // passes whose loads are in flight together
 
-// Work unit ("group") = one row x 4 consecutive K-blocks = 128 elements =
-// 16 lanes x 16 bytes, producing one 32-bit word of the scale layout.  A warp
-// handles two groups per step.  Groups cover the padded scale buffer, so the
-// padding words (rows >= rows, blocks >= k/32) are written as 0 here too.
+// One CTA per row of the padded scale buffer (grid-stride).  A "group" is one
+// row x 4 consecutive K-blocks = 128 elements = 16 lanes x 16 bytes and
+// produces one 32-bit word of the scale layout; a warp handles two groups per
+// pass and the CTA 16.  All loads of up to kQ2Passes passes are issued before
+// any arithmetic.  Rows >= rows and blocks >= k/32 (padding) get exponent 0.
 __global__ void __launch_bounds__(kQ2Threads) quant_mx_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
                                                               int64_t k, int64_t ld_x, uint8_t* __restrict__ q,
-                                                              int64_t ld_q, uint8_t* __restrict__ sf, int64_t n_kc,
-                                                              int64_t n_groups) {
+                                                              int64_t ld_q, uint8_t* __restrict__ sf, int n_kc,
+                                                              int64_t rows_pad) {
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4;    // which of the warp's two groups
-  const int sub = lane & 15;     // lane within the group
-  const int kb_in = sub >> 2;    // K-block within the group
-  const int v_in = sub & 3;      // 16-byte vector within the block
-  const int64_t nkb = k / 32;
-  const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t step = nwarps * 2;
-
-  for (int64_t g0 = warp_id * 2; g0 < n_groups; g0 += step * kQ2Unroll) {
-    uint4 v[kQ2Unroll];
-    int64_t row[kQ2Unroll], kb[kQ2Unroll], g[kQ2Unroll];
-    bool real[kQ2Unroll];
+  const int warp = threadIdx.x >> 5;
+  const int half = lane >> 4;        // which of the warp's two groups
+  const int sub = lane & 15;         // lane within the group
+  const int kb_in = sub >> 2;        // K-block within the group
+  const int v_in = sub & 3;          // 16-byte vector within the block
+  const int gid = warp * 2 + half;   // group within a pass
+  const int nkb = static_cast<int>(k / 32);
+  for (int64_t row = blockIdx.x; row < rows_pad; row += gridDim.x) {
+    const bool row_real = row < rows;
+    const __nv_bfloat16* xr = x + (row_real ? row : 0) * ld_x;
+    uint8_t* qr = q + (row_real ? row : 0) * ld_q;
+    uint8_t* sf_row = sf + (row / 128) * static_cast<int64_t>(n_kc) * 512 + (row % 32) * 16 + ((row % 128) / 32) * 4;
+    for (int kc0 = 0; kc0 < n_kc; kc0 += 16 * kQ2Passes) {
+      uint4 v[kQ2Passes];
 #pragma unroll
-    for (int u = 0; u < kQ2Unroll; ++u) {
-      g[u] = g0 + u * step + half;
-      const int64_t gg = g[u] < n_groups ? g[u] : 0;
-      row[u] = gg / n_kc;
-      kb[u] = (gg % n_kc) * 4 + kb_in;
-      real[u] = (g[u] < n_groups) && (row[u] < rows) && (kb[u] < nkb);
-      v[u] = real[u] ? ld_stream_16(x + row[u] * ld_x + kb[u] * 32 + v_in * 8) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < kQ2Unroll; ++u) {
-      float f[8];
-      bf16x8_to_f32(v[u], f);
-      float amax = absmax8(f);
-      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-      const int e = real[u] ? mx_exponent(amax) : 0;
-      if (real[u]) {
-        const float inv = mx_inv_scale(e);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] *= inv;  // exact: power-of-two scaling
-        *reinterpret_cast<uint2*>(q + row[u] * ld_q + kb[u] * 32 + v_in * 8) = f32x8_to_e4m3(f);
+      for (int ps = 0; ps < kQ2Passes; ++ps) {
+        const int kc = kc0 + ps * 16 + gid;
+        const int kb = kc * 4 + kb_in;
+        v[ps] = (row_real && kc < n_kc && kb < nkb) ? ld_stream_16(xr + kb * 32 + v_in * 8) : make_uint4(0, 0, 0, 0);
       }
-      // gather the group's four exponents into its first lane
-      const int base = half * 16;
-      const uint32_t e0 = __shfl_sync(0xFFFFFFFFu, e, base + 0);
-      const uint32_t e1 = __shfl_sync(0xFFFFFFFFu, e, base + 4);
-      const uint32_t e2 = __shfl_sync(0xFFFFFFFFu, e, base + 8);
-      const uint32_t e3 = __shfl_sync(0xFFFFFFFFu, e, base + 12);
-      if (sub == 0 && g[u] < n_groups) {
-        const int64_t r = row[u];
-        const int64_t kc = g[u] % n_kc;
-        const int64_t off = ((r / 128) * n_kc + kc) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4;
-        *reinterpret_cast<uint32_t*>(sf + off) = e0 | (e1 << 8) | (e2 << 16) | (e3 << 24);
+#pragma unroll
+      for (int ps = 0; ps < kQ2Passes; ++ps) {
+        if (kc0 + ps * 16 >= n_kc) break;  // the same for every thread of the CTA
+        const int kc = kc0 + ps * 16 + gid;
+        const int kb = kc * 4 + kb_in;
+        const bool real = row_real && kc < n_kc && kb < nkb;
+        float f[8];
+        bf16x8_to_f32(v[ps], f);
+        float amax = absmax8(f);
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+        const int e = real ? mx_exponent(amax) : 0;
+        if (real) {
+          const float inv = mx_inv_scale(e);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) f[j] *= inv;  // exact: power-of-two scaling
+          *reinterpret_cast<uint2*>(qr + kb * 32 + v_in * 8) = f32x8_to_e4m3(f);
+        }
+        // gather the group's four exponents into its first lane
+        const int base = half * 16;
+        const uint32_t e0 = __shfl_sync(0xFFFFFFFFu, e, base + 0);
+        const uint32_t e1 = __shfl_sync(0xFFFFFFFFu, e, base + 4);
+        const uint32_t e2 = __shfl_sync(0xFFFFFFFFu, e, base + 8);
+        const uint32_t e3 = __shfl_sync(0xFFFFFFFFu, e, base + 12);
+        if (sub == 0 && kc < n_kc)
+          *reinterpret_cast<uint32_t*>(sf_row + static_cast<int64_t>(kc) * 512) = e0 | (e1 << 8) | (e2 << 16) | (e3 << 24);
       }
     }
   }

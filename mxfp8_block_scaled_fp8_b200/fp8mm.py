@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libfp8mm.so")
 
 FP8MM_OK = 0
 FP8MM_ERR_DEVICE = 7
-KERNEL_AUTO, KERNEL_TILED, KERNEL_SMALL_M = 0, 1, 2
+KERNEL_AUTO, KERNEL_TILED, KERNEL_SMALL_M, KERNEL_TILED_1SM, KERNEL_TILED_2SM = 0, 1, 2, 3, 4
 
 
 class Fp8mmError(RuntimeError):
@@ -119,7 +119,7 @@ def fp8_quantize_rowwise(x: torch.Tensor, q: torch.Tensor | None = None, scale: 
 
 
 def fp8_gemm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
-             c: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+             c: torch.Tensor | None = None, kernel: int = KERNEL_AUTO, stream=None) -> torch.Tensor:
     """C bf16 [m, n] = diag(scale_a) (A x B^T) diag(scale_b); a [m,k], b [n,k] E4M3 codes."""
     a, b = _u8(a), _u8(b)
     _need(a, torch.uint8, "a"); _need(b, torch.uint8, "b")
@@ -130,8 +130,9 @@ def fp8_gemm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: t
         raise ValueError("a [m,k] and b [n,k] must be contiguous with the same k")
     if c is None:
         c = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
+    opts = Opts(None, 0, kernel, 0)
     _check("fp8_gemm", lib().fp8_gemm(a.data_ptr(), b.data_ptr(), m, n, k, scale_a.data_ptr(), scale_b.data_ptr(),
-                                      c.data_ptr(), _ld(c, "c"), None, _stream(stream)))
+                                      c.data_ptr(), _ld(c, "c"), ctypes.byref(opts), _stream(stream)))
     return c
 
 

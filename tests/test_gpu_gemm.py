@@ -31,14 +31,14 @@ def _rows_cols(m, n, nr, nc, seed):
     return rows, cols
 
 
-def run_rowwise(a_cpu, bt_cpu, sample=None, label=""):
+def run_rowwise(a_cpu, bt_cpu, sample=None, label="", kernel=fp8mm.KERNEL_AUTO):
     """Mode 1 end to end: quantize both operands per row, GEMM, compare."""
     import oracle as orc
     qa, sa = orc.quantize_rowwise(synthetic.bits(a_cpu))
     qb, sb = orc.quantize_rowwise(synthetic.bits(bt_cpu))
     ga, gsa = fp8mm.fp8_quantize_rowwise(gu.to_dev(a_cpu))
     gb, gsb = fp8mm.fp8_quantize_rowwise(gu.to_dev(bt_cpu))
-    c = fp8mm.fp8_gemm(ga, gb, gsa, gsb)
+    c = fp8mm.fp8_gemm(ga, gb, gsa, gsb, kernel=kernel)
     torch.cuda.synchronize()
     if sample is None:
         c_ref, bound = orc.gemm_rowwise(qa, qb, sa, sb)
@@ -76,14 +76,16 @@ def test_tiny_rowwise_full():
     run_rowwise(a, bt, label="tiny 128x256x512")
 
 
-def test_qk_mx_full():
+@pytest.mark.parametrize("kernel", [fp8mm.KERNEL_TILED_2SM, fp8mm.KERNEL_TILED_1SM], ids=["2sm", "1sm"])
+def test_qk_mx_full(kernel):
     a, bt = synthetic.qk()
-    run_mx(a, bt, label="qk 2048x1024x4096", kernel=fp8mm.KERNEL_TILED)
+    run_mx(a, bt, label="qk 2048x1024x4096", kernel=kernel)
 
 
-def test_attn_rowwise_sampled():
+@pytest.mark.parametrize("kernel", [fp8mm.KERNEL_AUTO, fp8mm.KERNEL_TILED_1SM], ids=["auto", "1sm"])
+def test_attn_rowwise_sampled(kernel):
     a, bt = synthetic.attn()
-    run_rowwise(a, bt, sample=_rows_cols(8192, 2048, 192, 64, 2), label="attn 8192x2048x8192")
+    run_rowwise(a, bt, sample=_rows_cols(8192, 2048, 192, 64, 2), label="attn 8192x2048x8192", kernel=kernel)
 
 
 def test_ffn_up_mx_sampled():
@@ -93,20 +95,25 @@ def test_ffn_up_mx_sampled():
 
 # ------------------------------------------------------------ shapes and edges
 
+KERNELS = pytest.mark.parametrize("kernel", [fp8mm.KERNEL_TILED_1SM, fp8mm.KERNEL_TILED_2SM], ids=["1sm", "2sm"])
+
+
+@KERNELS
 @pytest.mark.parametrize("m,n,k", [(1, 256, 512), (200, 136, 320), (129, 257, 160), (256, 512, 16),
-                                   (300, 1000, 1040), (128, 256, 128)])
-def test_rowwise_ragged(m, n, k):
+                                   (300, 1000, 1040), (128, 256, 128), (520, 264, 384)])
+def test_rowwise_ragged(m, n, k, kernel):
     a = synthetic.random_bf16((m, k), seed=m + 1)
     bt = synthetic.random_bf16((n, k), seed=n + 2)
-    run_rowwise(a, bt, label=f"rowwise {m}x{n}x{k}")
+    run_rowwise(a, bt, label=f"rowwise {m}x{n}x{k} kernel {kernel}", kernel=kernel)
 
 
+@KERNELS
 @pytest.mark.parametrize("m,n,k", [(65, 256, 512), (200, 136, 320), (129, 257, 96), (300, 1000, 1056),
-                                   (128, 128, 32), (1, 384, 256)])
-def test_mx_ragged_tiled(m, n, k):
+                                   (128, 128, 32), (1, 384, 256), (520, 264, 384)])
+def test_mx_ragged_tiled(m, n, k, kernel):
     a = synthetic.random_bf16((m, k), seed=m + 3)
     bt = synthetic.random_bf16((n, k), seed=n + 4, sigma=0.05)
-    run_mx(a, bt, label=f"mx {m}x{n}x{k}", kernel=fp8mm.KERNEL_TILED)
+    run_mx(a, bt, label=f"mx {m}x{n}x{k} kernel {kernel}", kernel=kernel)
 
 
 def test_unit_scales_selection_closed_form():
