@@ -76,9 +76,21 @@ typedef struct fp8mm_opts {
    * per SM) or FP8MM_KERNEL_TILED_2SM (256x256 tiles on 2-CTA clusters with
    * cta_group::2 MMAs; each CTA loads its own halves of A and B). */
   int32_t kernel;
-  /* Number of CTAs for the small-M kernel's stream-K split (0 = one per SM). */
+  /* Number of CTAs for the small-M kernel's stream-K split (0 = automatic:
+   * one per SM, but at least 4 K slabs of 128 per CTA). */
   int32_t small_m_ctas;
+  /* FP8MM_FLAG_* bits. */
+  uint32_t flags;
 } fp8mm_opts;
+
+/* The small-M kernel is launched with programmatic dependent launch: it may
+ * start while the preceding kernel on the stream is still running, and waits
+ * for it before reading a, sf_a or writing c / the workspace.  With this flag
+ * it also starts streaming b and sf_b (the weights) before that wait, which
+ * hides its start-up behind the preceding kernel.  Set it only when b and
+ * sf_b were complete before the preceding kernel started (e.g. weights
+ * quantized at load time); never when the preceding kernel writes them. */
+#define FP8MM_FLAG_WEIGHTS_READY 1u
 
 #define FP8MM_KERNEL_AUTO 0
 #define FP8MM_KERNEL_TILED 1

@@ -38,6 +38,7 @@ struct DecodeArgs {
   float* partials;     // [2 * G][kNM][128] fp32
   unsigned* tickets;   // [n_tiles], zero between calls
   uint64_t timeout_ns;
+  int prefetch_w;      // weights may be read before the preceding kernel ends
 };
 
 template <int kNM, int kStages>
@@ -105,6 +106,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int64_t u_begin = dec_unit_start(b, p);
   const int64_t u_end = dec_unit_start(b + 1, p);
   const int first_tile = static_cast<int>(u_begin / p.num_k);
+  griddep_launch_dependents();  // a following kernel launched the same way may start its prologue
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -135,33 +137,60 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
+    // The CTA's slabs in order: slab i is unit u_begin + i = (tile t, K slab
+    // kb).  When the caller vouches that the weights do not depend on the
+    // preceding kernel (prefetch_w), the weights of the first stages are
+    // requested before griddepcontrol.wait; the activation always after it.
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
-      bool ok = true;
-      for (int64_t u = u_begin; ok && u < u_end;) {
-        const int t = static_cast<int>(u / p.num_k);
-        const int kb0 = static_cast<int>(u % p.num_k);
-        const int kb1 = static_cast<int>(kb0 + (u_end - u) < p.num_k ? kb0 + (u_end - u) : p.num_k);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[stage], Cfg::kWBytes + Cfg::kXBytes + 1024u);
-          tma_load_2d(smem + Cfg::kOffW + stage * Cfg::kWBytes, &tmW, &full[stage], kb * 128, t * 128);
-          tma_load_2d(smem + Cfg::kOffX + stage * Cfg::kXBytes, &tmX, &full[stage], kb * 128, 0);
-          bulk_load(smem + Cfg::kOffSfw + stage * 512, p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u,
-                    &full[stage]);
-          bulk_load(smem + Cfg::kOffSfx + stage * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[stage]);
-          issued_mask |= 1u << stage;
-          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+      if (!p.prefetch_w) griddep_wait();
+      const int64_t nslabs = u_end - u_begin;
+      const int npre = static_cast<int>(nslabs < kStages ? nslabs : kStages);
+      const int t0 = static_cast<int>(u_begin / p.num_k);
+      const int kb0 = static_cast<int>(u_begin % p.num_k);
+      constexpr uint32_t kTx = Cfg::kWBytes + Cfg::kXBytes + 1024u;
+      int t = t0, kb = kb0;
+      for (int i = 0; i < npre; ++i) {  // fresh stages: nothing to wait for
+        mbar_arrive_expect_tx(&full[i], kTx);
+        tma_load_2d(smem + Cfg::kOffW + i * Cfg::kWBytes, &tmW, &full[i], kb * 128, t * 128);
+        bulk_load(smem + Cfg::kOffSfw + i * 512, p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u, &full[i]);
+        if (++kb == p.num_k) {
+          kb = 0;
+          ++t;
         }
-        u += kb1 - kb0;
+      }
+      griddep_wait();
+      t = t0;
+      kb = kb0;
+      for (int i = 0; i < npre; ++i) {
+        tma_load_2d(smem + Cfg::kOffX + i * Cfg::kXBytes, &tmX, &full[i], kb * 128, 0);
+        bulk_load(smem + Cfg::kOffSfx + i * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[i]);
+        if (++kb == p.num_k) {
+          kb = 0;
+          ++t;
+        }
+      }
+      int stage = npre % kStages;
+      uint32_t phase = (npre == kStages) ? 1u : 0u;
+      uint32_t issued_mask = (npre == kStages) ? ((1u << kStages) - 1u) : ((1u << npre) - 1u);
+      uint32_t issued_parity = 0;
+      for (int64_t i = npre; i < nslabs; ++i) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) break;
+        mbar_arrive_expect_tx(&full[stage], kTx);
+        tma_load_2d(smem + Cfg::kOffW + stage * Cfg::kWBytes, &tmW, &full[stage], kb * 128, t * 128);
+        tma_load_2d(smem + Cfg::kOffX + stage * Cfg::kXBytes, &tmX, &full[stage], kb * 128, 0);
+        bulk_load(smem + Cfg::kOffSfw + stage * 512, p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u,
+                  &full[stage]);
+        bulk_load(smem + Cfg::kOffSfx + stage * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[stage]);
+        issued_mask |= 1u << stage;
+        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        if (++kb == p.num_k) {
+          kb = 0;
+          ++t;
+        }
       }
       for (int s = 0; s < kStages; ++s)
         if (issued_mask & (1u << s))
@@ -216,6 +245,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------ epilogue
+    griddep_wait();  // the workspace and C may still be in use by the preceding kernel
     const int sp = warp & 3;
     const int nl = sp * 32 + lane;  // weight row inside the tile = output column
     int acc = 0;
@@ -276,16 +306,30 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       if (!epi_meet()) break;
       if (*last_flag) {
         __threadfence();
+        // Sum the contributors' partials in CTA order (fixed, so the result
+        // does not depend on arrival order); kU contributors' loads are in
+        // flight at a time.
+        constexpr int kU = kNM <= 16 ? 4 : (kNM <= 32 ? 2 : 1);
         float sum[kNM];
 #pragma unroll
         for (int j = 0; j < kNM; ++j) sum[j] = 0.f;
-        for (int bb = b_first; bb <= b_last; ++bb) {
-          const int first_bb = static_cast<int>(dec_unit_start(bb, p) / p.num_k);
-          const int sl = 2 * bb + (t == first_bb ? 0 : 1);
-          const float* src = p.partials + static_cast<int64_t>(sl) * kNM * 128;
+        for (int bb = b_first; bb <= b_last; bb += kU) {
+          float v[kU][kNM];
 #pragma unroll
-          for (int j = 0; j < kNM; ++j)
-            if (j < p.m) sum[j] += __ldcg(src + j * 128 + nl);
+          for (int q = 0; q < kU; ++q) {
+            const int b2 = bb + q;
+            const float* src = nullptr;
+            if (b2 <= b_last) {
+              const int first_b2 = static_cast<int>(dec_unit_start(b2, p) / p.num_k);
+              src = p.partials + static_cast<int64_t>(2 * b2 + (t == first_b2 ? 0 : 1)) * kNM * 128;
+            }
+#pragma unroll
+            for (int j = 0; j < kNM; ++j) v[q][j] = (src != nullptr && j < p.m) ? __ldcg(src + j * 128 + nl) : 0.f;
+          }
+#pragma unroll
+          for (int q = 0; q < kU; ++q)
+#pragma unroll
+            for (int j = 0; j < kNM; ++j) sum[j] += v[q][j];
         }
         if (n_col < p.n) {
 #pragma unroll

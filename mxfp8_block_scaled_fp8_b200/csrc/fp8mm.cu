@@ -133,6 +133,29 @@ static fp8mm_status make_sf_map(CUtensorMap* map, const void* sf, int64_t k, int
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Launch with programmatic stream serialisation (the kernel may begin while
+// the preceding kernel on the stream finishes; it waits for it in-kernel).
+template <typename... KArgs, typename... Args>
+static fp8mm_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                               Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess) {
+    t_last_cuda_error = static_cast<int>(e);
+    return FP8MM_ERR_LAUNCH;
+  }
+  return FP8MM_OK;
+}
+
 static fp8mm_status launched() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FP8MM_OK : cuda_fail(e);
@@ -141,7 +164,9 @@ static fp8mm_status launched() {
 // ------------------------------------------------------------------ kernels' configs
 using G1 = GemmCfg<false, 256, 4, 2>;
 using G2 = GemmCfg<true, 256, 4, 1>;
-constexpr int kDecStages = 8;
+// Small-M ring depth: as many stages as shared memory holds (the weight
+// stream needs ~25 MB in flight GPU-wide to cover the loaded HBM latency).
+constexpr int dec_stages(int nm) { return nm <= 16 ? 11 : nm <= 32 ? 10 : nm <= 48 ? 9 : 8; }
 
 __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
   __shared__ uint64_t bar;
@@ -295,15 +320,40 @@ static size_t small_m_partials_bytes(int ctas, int nm) {
   return (b + 255) & ~size_t(255);
 }
 
+// Launched with programmatic stream serialisation: the kernel may start while
+// the preceding kernel on the stream (normally the activation quantizer) is
+// still running; it prefetches weights and then waits for it in-kernel.
 template <int kNM>
 static fp8mm_status launch_small_m_t(const CUtensorMap& tw, const CUtensorMap& tx, const DecodeArgs& p,
                                      cudaStream_t stream, int dev) {
-  using Cfg = DecodeCfg<kNM, kDecStages>;
-  auto kern = gemm_small_m_kernel<kNM, kDecStages>;
+  constexpr int kStages = dec_stages(kNM);
+  using Cfg = DecodeCfg<kNM, kStages>;
+  auto kern = gemm_small_m_kernel<kNM, kStages>;
   fp8mm_status st = ensure_smem(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, dev);
   if (st != FP8MM_OK) return st;
-  kern<<<p.ctas, kDecThreads, Cfg::kSmemBytes, stream>>>(tw, tx, p);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(p.ctas, 1, 1);
+  cfg.blockDim = dim3(kDecThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, p);
+  if (e != cudaSuccess) return cuda_fail(e);
   return launched();
+}
+
+// CTAs of the small-M kernel: the requested number, else one per SM but no
+// fewer than 4 K slabs per CTA (more CTAs would only add partial tiles to
+// reduce); never more than there are slabs, never fewer than the tiles.
+constexpr int64_t kMinSlabsPerCta = 4;
+static int small_m_ctas(int64_t units, int64_t n_tiles, int64_t requested, int64_t sms) {
+  int64_t g = requested > 0 ? requested : std::min<int64_t>(sms, std::max<int64_t>(n_tiles, cdiv(units, kMinSlabsPerCta)));
+  g = std::min<int64_t>(g, units);
+  return static_cast<int>(std::max<int64_t>(g, 1));
 }
 
 static fp8mm_status launch_small_m(const void* a, const uint8_t* sfa, const void* b, const uint8_t* sfb, int64_t m,
@@ -323,12 +373,11 @@ static fp8mm_status launch_small_m(const void* a, const uint8_t* sfa, const void
   p.sfx = sfa;
   p.n_kc = p.num_k;
   p.timeout_ns = wait_timeout_ns();
+  p.prefetch_w = (opt != nullptr && (opt->flags & FP8MM_FLAG_WEIGHTS_READY)) ? 1 : 0;
   if (opt == nullptr || opt->workspace == nullptr) {
     p.ctas = p.n_tiles;  // one CTA per weight tile, whole K: no partial sums
   } else {
-    int64_t g = opt->small_m_ctas > 0 ? opt->small_m_ctas : dev.sms;
-    g = std::min<int64_t>(g, p.units);
-    p.ctas = static_cast<int>(std::max<int64_t>(g, 1));
+    p.ctas = small_m_ctas(p.units, p.n_tiles, opt->small_m_ctas, dev.sms);
     const size_t need = fp8mm_workspace_bytes(m, n, k, p.ctas);
     if (opt->workspace_bytes < need || !aligned(opt->workspace, 256)) return FP8MM_ERR_WORKSPACE;
     p.partials = static_cast<float*>(opt->workspace);
@@ -418,7 +467,7 @@ size_t fp8mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas) {
     cudaGetLastError();  // a host without a GPU leaves an error behind
   }
   const int64_t units = cdiv(n, 128) * cdiv(k, 128);
-  g = static_cast<int>(std::min<int64_t>(g, units));
+  g = small_m_ctas(units, cdiv(n, 128), ctas, g);
   const size_t tickets = static_cast<size_t>(cdiv(n, 128)) * sizeof(unsigned);
   return small_m_partials_bytes(g, small_m_tile(m)) + ((tickets + 255) & ~size_t(255));
 }
@@ -443,22 +492,20 @@ fp8mm_status fp8_quantize_rowwise(const void* x_bf16, int64_t rows, int64_t k, i
   const int64_t nvec = k / 8;
   if (nvec > static_cast<int64_t>(kQ1Threads) * 8) {
     const int grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(dev.sms) * 8));
-    quant_rowwise_2pass_kernel<<<grid, kQ1Threads, 0, s>>>(x, rows, k, ld_x, q, ld_q, scale);
-    return launched();
+    fp8mm_status st2 = launch_pdl(quant_rowwise_2pass_kernel, dim3(grid), dim3(kQ1Threads), 0, s, x, rows, k, ld_x,
+                                  q, ld_q, scale);
+    return st2 != FP8MM_OK ? st2 : launched();
   }
   const int threads = static_cast<int>(std::min<int64_t>(kQ1Threads, std::max<int64_t>(32, cdiv(nvec, 32) * 32)));
   const int64_t nv = cdiv(std::max<int64_t>(nvec, 1), threads);
   const int per_sm = 2048 / threads;
   const int grid = static_cast<int>(std::min<int64_t>(rows, static_cast<int64_t>(dev.sms) * per_sm));
-  if (nv <= 1)
-    quant_rowwise_kernel<1><<<grid, threads, 0, s>>>(x, rows, k, ld_x, q, ld_q, scale);
-  else if (nv <= 2)
-    quant_rowwise_kernel<2><<<grid, threads, 0, s>>>(x, rows, k, ld_x, q, ld_q, scale);
-  else if (nv <= 4)
-    quant_rowwise_kernel<4><<<grid, threads, 0, s>>>(x, rows, k, ld_x, q, ld_q, scale);
-  else
-    quant_rowwise_kernel<8><<<grid, threads, 0, s>>>(x, rows, k, ld_x, q, ld_q, scale);
-  return launched();
+  auto kern = nv <= 1 ? quant_rowwise_kernel<1>
+              : nv <= 2 ? quant_rowwise_kernel<2>
+              : nv <= 4 ? quant_rowwise_kernel<4>
+                        : quant_rowwise_kernel<8>;
+  st = launch_pdl(kern, dim3(grid), dim3(threads), 0, s, x, rows, k, ld_x, q, ld_q, scale);
+  return st != FP8MM_OK ? st : launched();
 }
 
 fp8mm_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, void* q_e4m3, int64_t ld_q,
@@ -474,10 +521,10 @@ fp8mm_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
   const int64_t n_kc = cdiv(k, 128);
   const int64_t rows_pad = cdiv(rows, 128) * 128;
   const int grid = static_cast<int>(std::min<int64_t>(rows_pad, static_cast<int64_t>(dev.sms) * 8));
-  quant_mx_kernel<<<grid, kQ2Threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x_bf16), rows, k, ld_x, static_cast<uint8_t*>(q_e4m3), ld_q, sf,
-      static_cast<int>(n_kc), rows_pad);
-  return launched();
+  st = launch_pdl(quant_mx_kernel, dim3(grid), dim3(kQ2Threads), 0, static_cast<cudaStream_t>(stream),
+                  static_cast<const __nv_bfloat16*>(x_bf16), rows, k, ld_x, static_cast<uint8_t*>(q_e4m3), ld_q, sf,
+                  static_cast<int>(n_kc), rows_pad);
+  return st != FP8MM_OK ? st : launched();
 }
 
 static fp8mm_status check_gemm_common(const void* a, const void* b, int64_t m, int64_t n, int64_t k, const void* c,

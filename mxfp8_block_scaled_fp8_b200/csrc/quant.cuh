@@ -10,12 +10,16 @@
 //   per 32 elements).
 //
 // Both kernels read bf16 with 16-byte vector loads and write E4M3 with
-// 8-byte stores; a warp always covers a contiguous run of one row.
+// 8-byte stores; a warp always covers a contiguous run of one row.  They are
+// launched with programmatic dependent launch and wait for the preceding
+// kernel before touching memory, so only their launch overlaps it.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cstdint>
+
+#include "ptx.cuh"
 
 namespace fp8mm {
 
@@ -69,6 +73,8 @@ __global__ void __launch_bounds__(kQ1Threads) quant_rowwise_kernel(const __nv_bf
   __shared__ float red[kQ1Threads / 32];
   const int nvec = static_cast<int>(k / 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_launch_dependents();
+  griddep_wait();  // x and the outputs may belong to the preceding kernel
   for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
     const __nv_bfloat16* xr = x + row * ld_x;
     uint4 v[NV];
@@ -117,6 +123,8 @@ __global__ void __launch_bounds__(kQ1Threads) quant_rowwise_2pass_kernel(const _
   __shared__ float red[kQ1Threads / 32];
   const int64_t nvec = k / 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_launch_dependents();
+  griddep_wait();
   for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
     const __nv_bfloat16* xr = x + row * ld_x;
     float amax = 0.f;
@@ -185,6 +193,8 @@ __global__ void __launch_bounds__(kQ2Threads) quant_mx_kernel(const __nv_bfloat1
   const int v_in = sub & 3;          // 16-byte vector within the block
   const int gid = warp * 2 + half;   // group within a pass
   const int nkb = static_cast<int>(k / 32);
+  griddep_launch_dependents();       // a following GEMM may start prefetching its weights
+  griddep_wait();                    // x and the outputs may belong to the preceding kernel
   for (int64_t row = blockIdx.x; row < rows_pad; row += gridDim.x) {
     const bool row_real = row < rows;
     const __nv_bfloat16* xr = x + (row_real ? row : 0) * ld_x;

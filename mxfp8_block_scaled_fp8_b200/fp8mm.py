@@ -35,9 +35,12 @@ class Fp8mmError(RuntimeError):
         super().__init__(msg)
 
 
+FLAG_WEIGHTS_READY = 1
+
+
 class Opts(ctypes.Structure):
     _fields_ = [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
-                ("kernel", ctypes.c_int32), ("small_m_ctas", ctypes.c_int32)]
+                ("kernel", ctypes.c_int32), ("small_m_ctas", ctypes.c_int32), ("flags", ctypes.c_uint32)]
 
 
 _lib = None
@@ -130,7 +133,7 @@ def fp8_gemm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: t
         raise ValueError("a [m,k] and b [n,k] must be contiguous with the same k")
     if c is None:
         c = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
-    opts = Opts(None, 0, kernel, 0)
+    opts = Opts(None, 0, kernel, 0, 0)
     _check("fp8_gemm", lib().fp8_gemm(a.data_ptr(), b.data_ptr(), m, n, k, scale_a.data_ptr(), scale_b.data_ptr(),
                                       c.data_ptr(), _ld(c, "c"), ctypes.byref(opts), _stream(stream)))
     return c
@@ -182,8 +185,10 @@ def workspace_bytes(m: int, n: int, k: int, ctas: int = 0) -> int:
 
 def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch.Tensor,
                c: torch.Tensor | None = None, workspace: torch.Tensor | None = None, kernel: int = KERNEL_AUTO,
-               small_m_ctas: int = 0, stream=None) -> torch.Tensor:
-    """C bf16 [m, n] = block-scaled A x B^T; a [m,k], b [n,k] codes with their library-layout scales."""
+               small_m_ctas: int = 0, weights_ready: bool = False, stream=None) -> torch.Tensor:
+    """C bf16 [m, n] = block-scaled A x B^T; a [m,k], b [n,k] codes with their library-layout scales.
+    weights_ready: b and sf_b were complete before the preceding kernel on the stream started (see
+    FP8MM_FLAG_WEIGHTS_READY)."""
     a, b = _u8(a), _u8(b)
     _need(a, torch.uint8, "a"); _need(b, torch.uint8, "b")
     _need(sf_a, torch.uint8, "sf_a"); _need(sf_b, torch.uint8, "sf_b")
@@ -195,7 +200,7 @@ def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch
         c = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
     opts = Opts(workspace.data_ptr() if workspace is not None else None,
                 workspace.numel() * workspace.element_size() if workspace is not None else 0,
-                kernel, small_m_ctas)
+                kernel, small_m_ctas, FLAG_WEIGHTS_READY if weights_ready else 0)
     _check("mxfp8_gemm", lib().mxfp8_gemm(a.data_ptr(), sf_a.data_ptr(), b.data_ptr(), sf_b.data_ptr(), m, n, k,
                                           c.data_ptr(), _ld(c, "c"), ctypes.byref(opts), _stream(stream)))
     return c

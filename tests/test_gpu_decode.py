@@ -45,12 +45,14 @@ def test_decode_sweep_stream_k(decode_data, name, m):
     qx, sfx = orc.mx_quantize(synthetic.bits(x))
     gx, gsfx = fp8mm.mxfp8_quantize(gu.to_dev(x))
     ws = _workspace(m, n, k)
-    c = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws)
+    # the weights were quantized long before: they may be streamed while the
+    # activation quantizer that precedes the GEMM is still running
+    c = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, weights_ready=True)
     torch.cuda.synchronize()
     c_ref, bound = orc.gemm_mx(qx, sfx, qw, sfw)
     gu.check_gemm(c, c_ref, bound, f"decode {name} m={m}")
     # counters are left at zero for the next call
-    c2 = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws)
+    c2 = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, weights_ready=True)
     torch.cuda.synchronize()
     assert torch.equal(c, c2), "second call with the same workspace differs"
 
@@ -93,6 +95,9 @@ def test_decode_partitions(decode_data, ctas):
 
 @pytest.mark.parametrize("m,n,k", [(3, 200, 96), (17, 130, 4128), (64, 384, 320), (33, 1000, 64)])
 def test_decode_ragged(m, n, k):
+    """Ragged shapes; the weights are quantized right before each GEMM on the
+    same stream, so the GEMM must not read them before that kernel ends
+    (no weights_ready flag)."""
     import oracle as orc
     x = synthetic.random_bf16((m, k), seed=m * 3 + k)
     w = synthetic.random_bf16((n, k), seed=n * 5 + k, sigma=0.02)
@@ -103,6 +108,7 @@ def test_decode_ragged(m, n, k):
     c_ref, bound = orc.gemm_mx(qx, sfx, qw, sfw)
     for ctas in (0, 5):
         ws = _workspace(m, n, k, ctas)
+        gw, gsfw = fp8mm.mxfp8_quantize(gu.to_dev(w))          # immediately precedes the GEMM
         c = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, small_m_ctas=ctas)
         torch.cuda.synchronize()
         gu.check_gemm(c, c_ref, bound, f"decode ragged {m}x{n}x{k} ctas={ctas}")
