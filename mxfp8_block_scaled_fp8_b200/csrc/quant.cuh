@@ -1,7 +1,7 @@
 // quant.cuh -- bf16 -> E4M3 quantizers for both scale modes (HBM-bound).
 //
 // Mode 1 (per row):  s = amax / 448 (IEEE fp32 division, 1 for a zero row),
-//   q = E4M3_RNE_sat(x / s).  Page "从 DeepGEMM 到 vLLM", listing 3
+//   q = E4M3_RNE_sat(x / s), x / s the correctly rounded fp32 quotient.  Page "从 DeepGEMM 到 vLLM", listing 3
 //   (_calibrate_scales) applied per row; listing 1 takes per-token scale_a
 //   and per-channel scale_b.
 // Mode 2 (MX, 1x32 blocks along K):  e = clamp(ceil(log2(amax/448)) + 127,
@@ -61,6 +61,28 @@ __device__ __forceinline__ uint2 f32x8_to_e4m3(const float (&y)[8]) {
 
 // ------------------------------------------------------------------ mode 1
 
+// x / s correctly rounded to fp32 without a division per element, by
+// Markstein's residual correction (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990): with r = RN(1/s) and q = RN(x r), the residual e = q s - x is exact
+// (one fma) and RN(q - e r) is RN(x / s).  For x with 8 significant bits (any
+// bf16 value) this holds for every pair of significands, which a host-side
+// test checks exhaustively with IEEE fp32 arithmetic; scaling by powers of two
+// keeps it while q, e and r stay in the normal range, which
+// quotient_fast_ok() ensures for every element that can give a nonzero code
+// (|x| >= 2^-102); smaller |x| give |x / s| < 2^-22 and the code 0 with the
+// sign of x either way.  The signs in the two fmas make x = -0 give -0.
+__device__ __forceinline__ float quotient_rn(float x, float s, float r) {
+  const float q = x * r;
+  const float e = __fmaf_rn(q, s, -x);
+  return __fmaf_rn(-e, r, q);
+}
+// Row scales for which quotient_rn() is exact: s in [2^-80, 2^126] (so r is
+// normal and every |x| >= 448 s 2^-11 exceeds 2^-102); other rows divide.
+__device__ __forceinline__ bool quotient_fast_ok(float s) {
+  return s >= 0x1p-80f && s <= 0x1p126f;
+}
+
 constexpr int kQ1Threads = 256;
 
 // One CTA per row (grid-stride over rows).  The row is held in registers
@@ -100,15 +122,30 @@ __global__ void __launch_bounds__(kQ1Threads) quant_rowwise_kernel(const __nv_bf
     const float s = (m == 0.f) ? 1.f : __fdiv_rn(m, 448.f);
     if (threadIdx.x == 0) scale[row] = s;
     uint8_t* qr = q + row * ld_q;
+    if (quotient_fast_ok(s)) {
+      const float r = __frcp_rn(s);
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int idx = threadIdx.x + i * blockDim.x;
-      if (idx < nvec) {
-        float f[8];
-        bf16x8_to_f32(v[i], f);
+      for (int i = 0; i < NV; ++i) {
+        const int idx = threadIdx.x + i * blockDim.x;
+        if (idx < nvec) {
+          float f[8];
+          bf16x8_to_f32(v[i], f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] = __fdiv_rn(f[j], s);
-        *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(idx) * 8) = f32x8_to_e4m3(f);
+          for (int j = 0; j < 8; ++j) f[j] = quotient_rn(f[j], s, r);
+          *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(idx) * 8) = f32x8_to_e4m3(f);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int idx = threadIdx.x + i * blockDim.x;
+        if (idx < nvec) {
+          float f[8];
+          bf16x8_to_f32(v[i], f);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) f[j] = __fdiv_rn(f[j], s);
+          *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(idx) * 8) = f32x8_to_e4m3(f);
+        }
       }
     }
   }
@@ -143,11 +180,13 @@ __global__ void __launch_bounds__(kQ1Threads) quant_rowwise_2pass_kernel(const _
     const float s = (m == 0.f) ? 1.f : __fdiv_rn(m, 448.f);
     if (threadIdx.x == 0) scale[row] = s;
     uint8_t* qr = q + row * ld_q;
+    const bool fast = quotient_fast_ok(s);
+    const float r = __frcp_rn(s);
     for (int64_t idx = threadIdx.x; idx < nvec; idx += blockDim.x) {
       float f[8];
       bf16x8_to_f32(*reinterpret_cast<const uint4*>(xr + idx * 8), f);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) f[j] = __fdiv_rn(f[j], s);
+      for (int j = 0; j < 8; ++j) f[j] = fast ? quotient_rn(f[j], s, r) : __fdiv_rn(f[j], s);
       *reinterpret_cast<uint2*>(qr + idx * 8) = f32x8_to_e4m3(f);
     }
   }

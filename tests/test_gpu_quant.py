@@ -162,6 +162,24 @@ def test_every_bf16_value_converts_like_the_oracle():
     _assert_rowwise(orc, x2, "all bf16 values, rowwise scale 1")
 
 
+def test_rowwise_many_scales_and_magnitudes():
+    """Per-row quotients x / s over many scales: each row's maximum is a random
+    bf16 over 2^-40..2^40 with a random mantissa, its other values spread
+    log-uniformly over 40 binades below it, so quotients fall in every E4M3
+    binade, the subnormal codes and below, and some lie next to rounding
+    midpoints; rows with subnormal or huge maxima are included."""
+    import oracle as orc
+    g = np.random.default_rng(77)
+    rows, k = 2048, 1024
+    amax = np.ldexp(1.0 + g.random(rows), g.integers(-40, 41, rows))
+    amax[:4] = [1e-39, 3e-36, 2.0 ** 126, 3.0e38]                # 1/s overflows; subnormal s; huge
+    mag = np.exp2(-40.0 * g.random((rows, k))) * amax[:, None]
+    x = np.where(g.random((rows, k)) < 0.5, -mag, mag)
+    x[np.arange(rows), g.integers(0, k, rows)] = amax           # the row maximum itself
+    xt = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+    _assert_rowwise(orc, xt, "rowwise many scales")
+
+
 def test_strided_input_rows():
     import oracle as orc
     base = synthetic.random_bf16((50, 640), seed=5)
