@@ -272,11 +272,18 @@ def _rows_measurements(fp8mm, synthetic, peaks, only=None):
             tg = _graph_time([lambda qw=qw, sfw=sfw: fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c, workspace=wsp,
                                                                       weights_ready=True)
                               for qw, sfw in wq])
+            # the same step as one launch: activation quantized inside the GEMM
+            wsq = torch.zeros(fp8mm.quantize_gemm_workspace_bytes(m, n, k), dtype=torch.uint8, device=dev)
+            tf_ = _graph_time([lambda qw=qw, sfw=sfw: fp8mm.mxfp8_quantize_gemm(x, qw, sfw, c, workspace=wsq,
+                                                                                weights_ready=True)
+                               for qw, sfw in wq])
             e2e_bytes = n * k + n * k / 32 + 2 * m * k + 2 * m * n
             gemm_bytes = n * k + n * k / 32 + m * k + 128 * k / 32 + 2 * m * n
             sweep[key] = {"ms": t, "GB/s": e2e_bytes / (t * 1e-3) / 1e9, "frac_hbm": e2e_bytes / (t * 1e-3) / 1e9 / hbm,
                           "gemm_ms": tg, "gemm_GB/s": gemm_bytes / (tg * 1e-3) / 1e9,
-                          "gemm_frac_hbm": gemm_bytes / (tg * 1e-3) / 1e9 / hbm}
+                          "gemm_frac_hbm": gemm_bytes / (tg * 1e-3) / 1e9 / hbm,
+                          "fused_ms": tf_, "fused_GB/s": e2e_bytes / (tf_ * 1e-3) / 1e9,
+                          "fused_frac_hbm": e2e_bytes / (tf_ * 1e-3) / 1e9 / hbm}
         del wq
     if sweep:
         out["decode"] = sweep

@@ -7,6 +7,6 @@ workload inputs.
 """
 from .fp8mm import (  # noqa: F401
     Fp8mmError, KERNEL_AUTO, KERNEL_SMALL_M, KERNEL_TILED, KERNEL_TILED_1SM, KERNEL_TILED_2SM, fp8_gemm, fp8_quantize_rowwise, last_device_error,
-    mxfp8_gemm, mxfp8_quantize, selftest_wait_timeout, sf_bytes, sf_from_canonical, sf_offset, sf_to_canonical,
-    version, workspace_bytes,
+    mxfp8_gemm, mxfp8_quantize, mxfp8_quantize_gemm, selftest_wait_timeout, sf_bytes, sf_from_canonical, sf_offset, sf_to_canonical,
+    quantize_gemm_workspace_bytes, version, workspace_bytes,
 )

@@ -13,16 +13,29 @@
 // arrival counter, and the last to arrive sums the partials in CTA order
 // (a fixed order, so results do not depend on timing), writes bf16 and
 // resets the counter.  No CTA ever waits for another.
+//
+// With kQX (m <= 16) the activation arrives as bf16 and is quantized inside
+// the kernel (the per-call activation quantization of page "[sglang]
+// FlashInfer v0.6.7 MXFP8 Gemm 통합", section 2, fused into the GEMM): four
+// more warps take the CTA's K slabs in turn (warp q the slabs q, q+4, ...).
+// Each TMA-loads its slabs of the raw activation (m rows x 128, zero past k)
+// into its own slots of a small ring, quantizes them with the 1x32 UE8M0 rule
+// of mxfp8_quantize (the same device functions, so codes and exponents are
+// identical), writes the E4M3 tile in the 128-byte-swizzled K-major layout the
+// MMA reads plus the exponents as the stage's scale chunk, and arrives on the
+// stage's full barrier next to the weight bytes.  The tile rows m..kNM-1 are
+// zeroed once and never written; K blocks past k quantize to zero with
+// exponent 127 and meet zero weights, so the output equals that of
+// mxfp8_quantize followed by the unfused kernel with the same CTA count.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace fp8mm {
-
-constexpr int kDecThreads = 192;
 
 struct DecodeArgs {
   int m, n, k;
@@ -39,25 +52,40 @@ struct DecodeArgs {
   unsigned* tickets;   // [n_tiles], zero between calls
   uint64_t timeout_ns;
   int prefetch_w;      // weights may be read before the preceding kernel ends
+  int raw_slots;       // kQX: raw activation slots in use (<= kMaxRawSlots)
+  uint32_t raw_bytes;  // kQX: bytes of one raw slab, m rows x 128 bf16
 };
 
-template <int kNM, int kStages>
+template <int kNM, int kStages, bool kQX = false>
 struct DecodeCfg {
   static_assert(kNM % 16 == 0 && kNM >= 16 && kNM <= 64, "token tile");
+  // warps: producer, MMA, four epilogue warps (+ four activation-quantizer warps)
+  static constexpr int kThreads = kQX ? 320 : 192;
+  static constexpr int kQuantWarp0 = 6;
   static constexpr int kWBytes = 128 * 128;
   static constexpr int kXBytes = kNM * 128;
+  // Raw activation ring: slabs of m rows x 128 bf16 (m * 256 bytes) in
+  // kRawRegion bytes; a multiple of 4 slots (slot i % R belongs to the warp
+  // of slab i), at most kMaxRawSlots.
+  static_assert(!kQX || kNM == 16, "activation quantized in the kernel for m <= 16");
+  static constexpr int kMaxRawSlots = kQX ? 16 : 0;
+  static constexpr int kRawRegion = kQX ? 32768 : 0;
   static constexpr int kOffW = 0;
   static constexpr int kOffX = kOffW + kStages * kWBytes;
   static constexpr int kOffSfw = kOffX + kStages * kXBytes;
   static constexpr int kOffSfx = kOffSfw + kStages * 512;
-  static constexpr int kOffBar = kOffSfx + kStages * 512;
-  static constexpr int kNumBars = 2 * kStages + 2 * 2 + 2;
+  static constexpr int kOffXRaw = kOffSfx + kStages * 512;
+  static constexpr int kOffBar = kOffXRaw + kRawRegion;
+  // full, empty per stage; acc_full, acc_empty x2; drain; epi_sync;
+  // with kQX: raw_full per raw slot
+  static constexpr int kNumBars = 2 * kStages + 2 * 2 + 2 + kMaxRawSlots;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static constexpr int kSfCol0 = 2 * kNM;
   static constexpr int kColsUsed = kSfCol0 + 8 * kStages;
   static constexpr int kTmemCols = kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128 : kColsUsed <= 256 ? 256 : 512;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kOffXRaw % 1024 == 0, "raw activation region 1024-byte aligned");
 };
 
 __device__ __forceinline__ int64_t dec_unit_start(int b, const DecodeArgs& p) {
@@ -83,11 +111,13 @@ __device__ __forceinline__ void regs_fence_16(uint32_t* r) {
                  "+r"(r[15]));
 }
 
-template <int kNM, int kStages>
-__global__ void __launch_bounds__(kDecThreads, 1)
+// tmX: the quantized activation (E4M3 [m, k], 128-byte swizzle, box 128 x
+// kNM), or with kQX the bf16 activation [m, k] (no swizzle, box 128 x kNM).
+template <int kNM, int kStages, bool kQX>
+__global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads, 1)
     gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                         const DecodeArgs p) {
-  using Cfg = DecodeCfg<kNM, kStages>;
+  using Cfg = DecodeCfg<kNM, kStages, kQX>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
@@ -96,6 +126,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint64_t* epi_sync = drain + 1;  // the four epilogue warps meet here (bounded)
+  uint64_t* raw_full = epi_sync + 1;  // kQX: raw activation slab landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 8);
@@ -110,7 +141,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], kQX ? 2 : 1);  // kQX: the weight bytes and the quantizer warp
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -119,6 +150,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     mbar_init(drain, 1);
     mbar_init(epi_sync, 4);
+    for (int j = 0; j < Cfg::kMaxRawSlots; ++j) mbar_init(&raw_full[j], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -147,7 +179,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int npre = static_cast<int>(nslabs < kStages ? nslabs : kStages);
       const int t0 = static_cast<int>(u_begin / p.num_k);
       const int kb0 = static_cast<int>(u_begin % p.num_k);
-      constexpr uint32_t kTx = Cfg::kWBytes + Cfg::kXBytes + 1024u;
+      constexpr uint32_t kTx = kQX ? Cfg::kWBytes + 512u : Cfg::kWBytes + Cfg::kXBytes + 1024u;
       int t = t0, kb = kb0;
       for (int i = 0; i < npre; ++i) {  // fresh stages: nothing to wait for
         mbar_arrive_expect_tx(&full[i], kTx);
@@ -162,8 +194,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       t = t0;
       kb = kb0;
       for (int i = 0; i < npre; ++i) {
-        tma_load_2d(smem + Cfg::kOffX + i * Cfg::kXBytes, &tmX, &full[i], kb * 128, 0);
-        bulk_load(smem + Cfg::kOffSfx + i * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[i]);
+        if (!kQX) {
+          tma_load_2d(smem + Cfg::kOffX + i * Cfg::kXBytes, &tmX, &full[i], kb * 128, 0);
+          bulk_load(smem + Cfg::kOffSfx + i * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[i]);
+        }
         if (++kb == p.num_k) {
           kb = 0;
           ++t;
@@ -177,10 +211,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) break;
         mbar_arrive_expect_tx(&full[stage], kTx);
         tma_load_2d(smem + Cfg::kOffW + stage * Cfg::kWBytes, &tmW, &full[stage], kb * 128, t * 128);
-        tma_load_2d(smem + Cfg::kOffX + stage * Cfg::kXBytes, &tmX, &full[stage], kb * 128, 0);
         bulk_load(smem + Cfg::kOffSfw + stage * 512, p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u,
                   &full[stage]);
-        bulk_load(smem + Cfg::kOffSfx + stage * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[stage]);
+        if (!kQX) {
+          tma_load_2d(smem + Cfg::kOffX + stage * Cfg::kXBytes, &tmX, &full[stage], kb * 128, 0);
+          bulk_load(smem + Cfg::kOffSfx + stage * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[stage]);
+        }
         issued_mask |= 1u << stage;
         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == kStages) {
@@ -243,7 +279,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mbar_wait(drain, 0, p.timeout_ns, nullptr, kSiteDrain);
     }
     __syncwarp();
-  } else {
+  } else if (warp < Cfg::kQuantWarp0) {
     // ------------------------------------------------------ epilogue
     griddep_wait();  // the workspace and C may still be in use by the preceding kernel
     const int sp = warp & 3;
@@ -338,6 +374,91 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
         if (threadIdx.x == 64) p.tickets[t] = 0u;
       }
+    }
+  } else if (kQX) {
+    // ------------------------------------------------------ activation quantizer
+    // Warp qw takes slabs qw, qw + 4, ...; its lane L handles the 16-byte
+    // vector v16 = L % 16 of rows L/16 + 2j < m: K block v16/4, so a block's
+    // four vectors sit in four adjacent lanes of one half-warp and its
+    // maximum is a two-step xor shuffle within that half.
+    const int qw = warp - Cfg::kQuantWarp0;
+    const int v16 = lane & 15;
+    const int kblk = v16 >> 2;
+    const unsigned half_mask = (lane & 16) ? 0xFFFF0000u : 0x0000FFFFu;
+    const int64_t nslabs = u_end - u_begin;
+    const int R = p.raw_slots;  // multiple of 4: slot i % R holds only this warp's slabs
+    const uint32_t raw_bytes = p.raw_bytes;
+    uint8_t* raw_base = smem + Cfg::kOffXRaw;
+    auto slab_kb = [&](int64_t i) { return static_cast<int>((u_begin + i) % p.num_k); };
+    auto load_raw = [&](int64_t i) {
+      const int slot = static_cast<int>(i % R);
+      mbar_arrive_expect_tx(&raw_full[slot], raw_bytes);
+      tma_load_2d(raw_base + slot * raw_bytes, &tmX, &raw_full[slot], slab_kb(i) * 128, 0);
+    };
+    // Tile rows m..kNM-1 (and their scale words, with the words of rows
+    // kNM..127 that the MMA never reads) are zeroed once; the loop below
+    // writes only rows < m.  Word (L, g) of a scale chunk holds row 32g + L.
+    const int qt = threadIdx.x - Cfg::kQuantWarp0 * 32;
+    for (int o = qt; o < kStages * (kNM - p.m) * 8; o += 128) {
+      const int st = o / ((kNM - p.m) * 8), rem = o % ((kNM - p.m) * 8);
+      reinterpret_cast<uint4*>(smem + Cfg::kOffX + st * Cfg::kXBytes + (p.m + rem / 8) * 128)[rem % 8] =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int w = qt; w < kStages * 128; w += 128) {
+      const int L = (w & 127) >> 2, g = w & 3;
+      if (32 * g + L >= p.m) reinterpret_cast<uint32_t*>(smem + Cfg::kOffSfx)[(w >> 7) * 128 + L * 4 + g] = 0u;
+    }
+    // The zeroed rows are read by the tensor core: each thread fences its
+    // stores to the async proxy, and the four warps meet before any of them
+    // arrives on a stage's full barrier.
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    griddep_wait();  // the activation may be written by the preceding kernel
+    int64_t issued = qw;  // next slab of this warp to load
+    if (lane == 0)
+      for (; issued < R && issued < nslabs; issued += 4) load_raw(issued);
+    bool ok = true;
+    int64_t i = qw;
+    for (; i < nslabs; i += 4) {
+      const int slot = static_cast<int>(i % R);
+      const int stage = static_cast<int>(i % kStages);
+      ok = ok && mbar_wait(&raw_full[slot], static_cast<uint32_t>((i / R) & 1), p.timeout_ns, abort_flag,
+                           kSiteQuantRaw);
+      ok = ok && mbar_wait(&empty[stage], static_cast<uint32_t>(((i / kStages) & 1) ^ 1), p.timeout_ns, abort_flag,
+                           kSiteQuantStage);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      const uint8_t* raw = raw_base + slot * raw_bytes;
+      uint8_t* xq = smem + Cfg::kOffX + stage * Cfg::kXBytes;
+      uint8_t* sfx = smem + Cfg::kOffSfx + stage * 512;
+#pragma unroll 2
+      for (int r = lane >> 4; r < p.m; r += 2) {
+        float f[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(raw + r * 256 + v16 * 16), f);
+        float a = absmax8(f);
+        a = fmaxf(a, __shfl_xor_sync(half_mask, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(half_mask, a, 2));
+        const int e = mx_exponent(a);
+        const float inv = mx_inv_scale(e);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] *= inv;
+        // byte v16*8 of row r: 16-byte chunk v16/2, stored at chunk (v16/2) ^ (r % 8)
+        *reinterpret_cast<uint2*>(xq + r * 128 + (((v16 >> 1) ^ (r & 7)) << 4) + (v16 & 1) * 8) = f32x8_to_e4m3(f);
+        if ((v16 & 3) == 0) sfx[(r & 31) * 16 + ((r & 127) >> 5) * 4 + kblk] = static_cast<uint8_t>(e);
+      }
+      fence_proxy_async_smem();  // the tile and scales are read by the tensor core (async proxy)
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&full[stage]);
+        if (issued < nslabs) {  // the slot's raw data is consumed: load this warp's next slab into it
+          load_raw(issued);
+          issued += 4;
+        }
+      }
+    }
+    // after an early exit, let raw loads still in flight land before the CTA ends
+    if (lane == 0) {
+      for (int64_t j = i; j < issued; j += 4)
+        mbar_wait(&raw_full[j % R], static_cast<uint32_t>((j / R) & 1), p.timeout_ns, nullptr, kSiteQuantDrain);
     }
   }
 

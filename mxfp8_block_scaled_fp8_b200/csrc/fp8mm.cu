@@ -112,6 +112,23 @@ static fp8mm_status make_map(CUtensorMap* map, const void* base, int64_t k, int6
   return FP8MM_OK;
 }
 
+// 2-D map over a row-major bf16 matrix [rows, k] with row stride ld elements,
+// box = 128 elements of K x box_rows rows, no swizzle, zero fill outside.
+static fp8mm_status make_map_bf16(CUtensorMap* map, const void* base, int64_t k, int64_t rows, int64_t ld,
+                                  int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2u};
+  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return FP8MM_OK;
+}
+
 // 3-D map over a library scale buffer viewed as uint32 [n_rt][n_kc][128]
 // (one 512-byte chunk per 128-row tile and 4-block group); box = box_rt chunks
 // of consecutive row tiles at one K group; zero fill past the last row tile.
@@ -167,6 +184,9 @@ using G2 = GemmCfg<true, 256, 4, 1>;
 // Small-M ring depth: as many stages as shared memory holds (the weight
 // stream needs ~25 MB in flight GPU-wide to cover the loaded HBM latency).
 constexpr int dec_stages(int nm) { return nm <= 16 ? 11 : nm <= 32 ? 10 : nm <= 48 ? 9 : 8; }
+// With the activation quantized in the kernel (m <= 16), its raw slabs take
+// shared memory too.
+constexpr int dec_stages_qx(int nm) { return nm <= 16 ? 10 : 0; }
 
 __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
   __shared__ uint64_t bar;
@@ -323,12 +343,12 @@ static size_t small_m_partials_bytes(int ctas, int nm) {
 // Launched with programmatic stream serialisation: the kernel may start while
 // the preceding kernel on the stream (normally the activation quantizer) is
 // still running; it prefetches weights and then waits for it in-kernel.
-template <int kNM>
+template <int kNM, bool kQX = false>
 static fp8mm_status launch_small_m_t(const CUtensorMap& tw, const CUtensorMap& tx, const DecodeArgs& p,
                                      cudaStream_t stream, int dev) {
-  constexpr int kStages = dec_stages(kNM);
-  using Cfg = DecodeCfg<kNM, kStages>;
-  auto kern = gemm_small_m_kernel<kNM, kStages>;
+  constexpr int kStages = kQX ? dec_stages_qx(kNM) : dec_stages(kNM);
+  using Cfg = DecodeCfg<kNM, kStages, kQX>;
+  auto kern = gemm_small_m_kernel<kNM, kStages, kQX>;
   fp8mm_status st = ensure_smem(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, dev);
   if (st != FP8MM_OK) return st;
   cudaLaunchConfig_t cfg = {};
@@ -336,7 +356,7 @@ static fp8mm_status launch_small_m_t(const CUtensorMap& tw, const CUtensorMap& t
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(p.ctas, 1, 1);
-  cfg.blockDim = dim3(kDecThreads, 1, 1);
+  cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = stream;
   cfg.attrs = attr;
@@ -356,9 +376,11 @@ static int small_m_ctas(int64_t units, int64_t n_tiles, int64_t requested, int64
   return static_cast<int>(std::max<int64_t>(g, 1));
 }
 
+// a: E4M3 codes [m, k] with scales sfa, or (qx) bf16 [m, k] with row stride
+// lda elements, quantized in the kernel (sfa unused).
 static fp8mm_status launch_small_m(const void* a, const uint8_t* sfa, const void* b, const uint8_t* sfb, int64_t m,
                                    int64_t n, int64_t k, void* c, int64_t ldc, const fp8mm_opts* opt,
-                                   cudaStream_t stream, const DeviceInfo& dev) {
+                                   cudaStream_t stream, const DeviceInfo& dev, bool qx = false, int64_t lda = 0) {
   const int nm = small_m_tile(m);
   DecodeArgs p{};
   p.m = static_cast<int>(m);
@@ -387,8 +409,14 @@ static fp8mm_status launch_small_m(const void* a, const uint8_t* sfa, const void
   CUtensorMap tw, tx;
   fp8mm_status st = make_map(&tw, b, k, n, 128);
   if (st != FP8MM_OK) return st;
-  st = make_map(&tx, a, k, m, nm);
+  st = qx ? make_map_bf16(&tx, a, k, m, lda, static_cast<int>(m)) : make_map(&tx, a, k, m, nm);
   if (st != FP8MM_OK) return st;
+  if (qx) {  // m <= 16: raw activation slabs of m rows x 128 bf16, a multiple of 4 slots
+    constexpr int kRegion = DecodeCfg<16, dec_stages_qx(16), true>::kRawRegion;
+    p.raw_bytes = static_cast<uint32_t>(m) * 256u;
+    p.raw_slots = static_cast<int>(std::min<int64_t>(16, kRegion / p.raw_bytes)) & ~3;
+    return launch_small_m_t<16, true>(tw, tx, p, stream, dev.device);
+  }
   switch (nm) {
     case 16: return launch_small_m_t<16>(tw, tx, p, stream, dev.device);
     case 32: return launch_small_m_t<32>(tw, tx, p, stream, dev.device);
@@ -580,6 +608,50 @@ fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e
   const bool pair = (kind == FP8MM_KERNEL_TILED_2SM) || (kind != FP8MM_KERNEL_TILED_1SM && m >= 256);
   if (pair) return launch_pair(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev);
   return launch_tiled(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev);
+}
+
+// Largest m whose activation is quantized inside the small-M kernel; above it
+// the per-CTA re-quantization of every K slab costs more than a separate
+// quantizer launch, which then writes into the workspace.
+constexpr int64_t kQuantInKernelMaxM = 16;
+
+static size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+size_t fp8mm_quantize_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas) {
+  if (m <= 0 || n <= 0 || k <= 0 || m > 64) return 0;
+  const size_t gemm = fp8mm_workspace_bytes(m, n, k, ctas);
+  if (m <= kQuantInKernelMaxM) return gemm;
+  return gemm + align256(static_cast<size_t>(m * k)) + align256(fp8mm_sf_bytes(m, k));
+}
+
+fp8mm_status mxfp8_quantize_gemm(const void* a_bf16, int64_t lda, const void* b_e4m3, const uint8_t* sf_b,
+                                 int64_t m, int64_t n, int64_t k, void* c_bf16, int64_t ldc, const fp8mm_opts* opt,
+                                 void* stream) {
+  if (m > 64) return FP8MM_ERR_SHAPE;
+  fp8mm_status st = check_gemm_common(a_bf16, b_e4m3, m, n, k, c_bf16, ldc, 32);
+  if (st != FP8MM_OK || m == 0 || n == 0) return st;
+  if (k > 0 && (lda < k || lda % 8 != 0)) return lda < k ? FP8MM_ERR_SHAPE : FP8MM_ERR_ALIGN;
+  if (k > 0 && sf_b == nullptr) return FP8MM_ERR_NULL;
+  if (!aligned(sf_b, 16)) return FP8MM_ERR_ALIGN;
+  const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
+  if (kind != FP8MM_KERNEL_AUTO && kind != FP8MM_KERNEL_SMALL_M) return FP8MM_ERR_SHAPE;
+  if (m > kQuantInKernelMaxM) {  // the quantized activation goes to the workspace tail
+    if (opt == nullptr || opt->workspace == nullptr) return FP8MM_ERR_WORKSPACE;
+    if (opt->workspace_bytes < fp8mm_quantize_gemm_workspace_bytes(m, n, k, opt->small_m_ctas) ||
+        !aligned(opt->workspace, 256))
+      return FP8MM_ERR_WORKSPACE;
+  }
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != FP8MM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (k == 0) return zero_output(c_bf16, m, n, ldc, s);
+  if (m <= kQuantInKernelMaxM)
+    return launch_small_m(a_bf16, nullptr, b_e4m3, sf_b, m, n, k, c_bf16, ldc, opt, s, dev, true, lda);
+  uint8_t* tail = static_cast<uint8_t*>(opt->workspace) + fp8mm_workspace_bytes(m, n, k, opt->small_m_ctas);
+  uint8_t* xq = tail;
+  uint8_t* sfx = tail + align256(static_cast<size_t>(m * k));
+  if ((st = mxfp8_quantize(a_bf16, m, k, lda, xq, k, sfx, stream)) != FP8MM_OK) return st;
+  return launch_small_m(xq, sfx, b_e4m3, sf_b, m, n, k, c_bf16, ldc, opt, s, dev);
 }
 
 unsigned int fp8mm_last_device_error(void) {

@@ -20,8 +20,8 @@ enum DevErr : unsigned { kDevErrTimeout = 1 };
 
 enum WaitSite : unsigned {
   kSiteProducerEmpty = 1, kSiteMmaFull = 2, kSiteMmaAccEmpty = 3, kSiteEpiAccFull = 4,
-  kSiteDrain = 5, kSiteProducerDrain = 6, kSiteSelfTest = 7, kSiteEpiSync = 8, kSiteSfFull = 9,
-  kSiteSfReady = 10,
+  kSiteDrain = 5, kSiteProducerDrain = 6, kSiteSelfTest = 7, kSiteEpiSync = 8, kSiteQuantRaw = 9,
+  kSiteQuantStage = 10, kSiteQuantDrain = 11,
 };
 
 __device__ __forceinline__ void record_error(unsigned kind, unsigned site) {
@@ -307,30 +307,6 @@ __device__ __forceinline__ void tmem_cp_32x128b_warpx4_pair(uint32_t taddr, uint
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-
-// Local (non-pair) 3-D tiled TMA load completing on this CTA's barrier.
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y,
-                                            int32_t z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-__device__ __forceinline__ uint4 ld_shared_16(const void* p) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(smem_u32(p)));
-  return v;
-}
-// Each thread writes 4 consecutive 32-bit columns of its own TMEM lane.
-__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint4& v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v.x), "r"(v.y),
-               "r"(v.z), "r"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 #define FP8MM_R32(r)                                                                                       \
   "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),          \

@@ -51,11 +51,13 @@ _SIGNATURES = {
     "mxfp8_quantize": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P], ctypes.c_int),
     "fp8_gemm": ([_P, _P, _I64, _I64, _I64, _P, _P, _P, _I64, ctypes.POINTER(Opts), _P], ctypes.c_int),
     "mxfp8_gemm": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, ctypes.POINTER(Opts), _P], ctypes.c_int),
+    "mxfp8_quantize_gemm": ([_P, _I64, _P, _P, _I64, _I64, _I64, _P, _I64, ctypes.POINTER(Opts), _P], ctypes.c_int),
     "fp8mm_sf_bytes": ([_I64, _I64], ctypes.c_size_t),
     "fp8mm_sf_offset": ([_I64, _I64, _I64, _I64], ctypes.c_int64),
     "fp8mm_sf_to_canonical": ([_P, _I64, _I64, _P], ctypes.c_int),
     "fp8mm_sf_from_canonical": ([_P, _I64, _I64, _P], ctypes.c_int),
     "fp8mm_workspace_bytes": ([_I64, _I64, _I64, ctypes.c_int32], ctypes.c_size_t),
+    "fp8mm_quantize_gemm_workspace_bytes": ([_I64, _I64, _I64, ctypes.c_int32], ctypes.c_size_t),
     "fp8mm_status_str": ([ctypes.c_int], ctypes.c_char_p),
     "fp8mm_last_cuda_error": ([], ctypes.c_int),
     "fp8mm_last_device_error": ([], ctypes.c_uint),
@@ -183,6 +185,10 @@ def workspace_bytes(m: int, n: int, k: int, ctas: int = 0) -> int:
     return int(lib().fp8mm_workspace_bytes(m, n, k, ctas))
 
 
+def quantize_gemm_workspace_bytes(m: int, n: int, k: int, ctas: int = 0) -> int:
+    return int(lib().fp8mm_quantize_gemm_workspace_bytes(m, n, k, ctas))
+
+
 def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch.Tensor,
                c: torch.Tensor | None = None, workspace: torch.Tensor | None = None, kernel: int = KERNEL_AUTO,
                small_m_ctas: int = 0, weights_ready: bool = False, stream=None) -> torch.Tensor:
@@ -203,6 +209,29 @@ def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch
                 kernel, small_m_ctas, FLAG_WEIGHTS_READY if weights_ready else 0)
     _check("mxfp8_gemm", lib().mxfp8_gemm(a.data_ptr(), sf_a.data_ptr(), b.data_ptr(), sf_b.data_ptr(), m, n, k,
                                           c.data_ptr(), _ld(c, "c"), ctypes.byref(opts), _stream(stream)))
+    return c
+
+
+def mxfp8_quantize_gemm(a: torch.Tensor, b: torch.Tensor, sf_b: torch.Tensor, c: torch.Tensor | None = None,
+                        workspace: torch.Tensor | None = None, kernel: int = KERNEL_AUTO, small_m_ctas: int = 0,
+                        weights_ready: bool = False, stream=None) -> torch.Tensor:
+    """C bf16 [m, n] = mxfp8_gemm(mxfp8_quantize(a), b) for m <= 64 from the bf16 activation a [m, k]:
+    quantized inside the GEMM kernel for m <= 16, else by its own launch into the workspace tail
+    (workspace of quantize_gemm_workspace_bytes(m, n, k, small_m_ctas) bytes, required for m > 16)."""
+    b = _u8(b)
+    _need(a, torch.bfloat16, "a"); _need(b, torch.uint8, "b"); _need(sf_b, torch.uint8, "sf_b")
+    m, k = a.shape
+    n = b.shape[0]
+    if b.shape[1] != k or not b.is_contiguous():
+        raise ValueError("b [n,k] must be contiguous with the k of a")
+    if c is None:
+        c = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
+    opts = Opts(workspace.data_ptr() if workspace is not None else None,
+                workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                kernel, small_m_ctas, FLAG_WEIGHTS_READY if weights_ready else 0)
+    _check("mxfp8_quantize_gemm", lib().mxfp8_quantize_gemm(
+        a.data_ptr(), _ld(a, "a"), b.data_ptr(), sf_b.data_ptr(), m, n, k, c.data_ptr(), _ld(c, "c"),
+        ctypes.byref(opts), _stream(stream)))
     return c
 
 
