@@ -180,8 +180,8 @@ fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e
  * mxfp8_quantize(a) followed by mxfp8_gemm(...) with the small-M kernel and
  * the same options, bit for bit (page "[sglang] FlashInfer v0.6.7 MXFP8 Gemm
  * 통합", section 2: the activation is quantized per call, the weights once).
- * For m <= 16 the activation is quantized inside the GEMM kernel: one launch
- * and no intermediate E4M3 activation in memory.  For 16 < m <= 64 the
+ * For m <= 8 the activation is quantized inside the GEMM kernel: one launch
+ * and no intermediate E4M3 activation in memory.  For 8 < m <= 64 the
  * quantizer runs as its own launch into the tail of the workspace, which is
  * then required.
  *   a_bf16  [m, k] bf16 activation, row stride lda elements (16-byte aligned,
@@ -189,7 +189,7 @@ fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e
  *   b_e4m3, sf_b, c_bf16, ldc, opt, stream: as for mxfp8_gemm (opt->kernel
  *           must be FP8MM_KERNEL_AUTO or FP8MM_KERNEL_SMALL_M; small_m_ctas
  *           and FP8MM_FLAG_WEIGHTS_READY act as there)
- *   opt->workspace: optional for m <= 16 (as for mxfp8_gemm); for m > 16 at
+ *   opt->workspace: optional for m <= 8 (as for mxfp8_gemm); for m > 8 at
  *           least fp8mm_quantize_gemm_workspace_bytes(m, n, k, small_m_ctas)
  *           bytes, 256-byte aligned (FP8MM_ERR_WORKSPACE otherwise)
  * Requires 0 <= m <= 64 and k % 32 == 0 (FP8MM_ERR_SHAPE otherwise).
@@ -198,7 +198,7 @@ fp8mm_status mxfp8_quantize_gemm(const void* a_bf16, int64_t lda, const void* b_
                                  int64_t m, int64_t n, int64_t k, void* c_bf16, int64_t ldc, const fp8mm_opts* opt,
                                  void* stream);
 /* Workspace bytes mxfp8_quantize_gemm needs: fp8mm_workspace_bytes(m, n, k,
- * ctas), plus for m > 16 room for the quantized activation and its scales
+ * ctas), plus for m > 8 room for the quantized activation and its scales
  * (each 256-byte aligned).  0 for m outside [1, 64]. */
 size_t fp8mm_quantize_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas);
 

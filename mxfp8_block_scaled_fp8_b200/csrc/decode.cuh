@@ -14,19 +14,22 @@
 // (a fixed order, so results do not depend on timing), writes bf16 and
 // resets the counter.  No CTA ever waits for another.
 //
-// With kQX (m <= 16) the activation arrives as bf16 and is quantized inside
+// With kQX (m <= 8) the activation arrives as bf16 and is quantized inside
 // the kernel (the per-call activation quantization of page "[sglang]
-// FlashInfer v0.6.7 MXFP8 Gemm 통합", section 2, fused into the GEMM): four
-// more warps take the CTA's K slabs in turn (warp q the slabs q, q+4, ...).
-// Each TMA-loads its slabs of the raw activation (m rows x 128, zero past k)
-// into its own slots of a small ring, quantizes them with the 1x32 UE8M0 rule
-// of mxfp8_quantize (the same device functions, so codes and exponents are
-// identical), writes the E4M3 tile in the 128-byte-swizzled K-major layout the
-// MMA reads plus the exponents as the stage's scale chunk, and arrives on the
-// stage's full barrier next to the weight bytes.  The tile rows m..kNM-1 are
-// zeroed once and never written; K blocks past k quantize to zero with
-// exponent 127 and meet zero weights, so the output equals that of
-// mxfp8_quantize followed by the unfused kernel with the same CTA count.
+// FlashInfer v0.6.7 MXFP8 Gemm 통합", section 2, fused into the GEMM): two
+// more warps take the CTA's K slabs in turn (warp q the slabs q, q+2, ...).
+// Each reads its slab of the activation (m rows x 128, zero past k) straight
+// from global memory -- it is small and shared by all CTAs, so it stays in L2
+// -- holding the next slab's loads in registers while it quantizes the
+// current one, one 32-element block per lane, with the 1x32 UE8M0 rule of
+// mxfp8_quantize (the same exponent and conversion functions, and the exact
+// block maximum, so codes and exponents are identical).  It writes the E4M3 tile
+// in the 128-byte-swizzled K-major layout the MMA reads plus the exponents as
+// the stage's scale chunk, and arrives on the stage's full barrier next to
+// the weight bytes.  The tile rows m..kNM-1 are zeroed once and never
+// written; K blocks past k quantize to zero with exponent 127 and meet zero
+// weights, so the output equals that of mxfp8_quantize followed by the
+// unfused kernel with the same CTA count.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -52,40 +55,37 @@ struct DecodeArgs {
   unsigned* tickets;   // [n_tiles], zero between calls
   uint64_t timeout_ns;
   int prefetch_w;      // weights may be read before the preceding kernel ends
-  int raw_slots;       // kQX: raw activation slots in use (<= kMaxRawSlots)
-  uint32_t raw_bytes;  // kQX: bytes of one raw slab, m rows x 128 bf16
+  const __nv_bfloat16* x;  // kQX: bf16 activation [m, k]
+  int64_t ldx;             // kQX: its row stride in elements
 };
 
 template <int kNM, int kStages, bool kQX = false>
 struct DecodeCfg {
   static_assert(kNM % 16 == 0 && kNM >= 16 && kNM <= 64, "token tile");
-  // warps: producer, MMA, four epilogue warps (+ four activation-quantizer warps)
-  static constexpr int kThreads = kQX ? 320 : 192;
+  // warps: producer, MMA, four epilogue warps (+ two activation-quantizer warps)
+  static constexpr int kQuantWarps = kQX ? 2 : 0;
+  static constexpr int kThreads = 192 + 32 * kQuantWarps;
   static constexpr int kQuantWarp0 = 6;
+  // Token tiles up to 32 keep shared memory and registers within half an SM,
+  // so the next kernel on the stream (launched early, programmatically) can
+  // hold a CTA on each SM and start streaming while this one finishes.
+  static constexpr int kMinBlocksPerSm = kNM <= 32 ? 2 : 1;
   static constexpr int kWBytes = 128 * 128;
   static constexpr int kXBytes = kNM * 128;
-  // Raw activation ring: slabs of m rows x 128 bf16 (m * 256 bytes) in
-  // kRawRegion bytes; a multiple of 4 slots (slot i % R belongs to the warp
-  // of slab i), at most kMaxRawSlots.
-  static_assert(!kQX || kNM == 16, "activation quantized in the kernel for m <= 16");
-  static constexpr int kMaxRawSlots = kQX ? 16 : 0;
-  static constexpr int kRawRegion = kQX ? 32768 : 0;
+  static_assert(!kQX || kNM == 16, "activation quantized in the kernel for m <= 8 (16-token tile)");
   static constexpr int kOffW = 0;
   static constexpr int kOffX = kOffW + kStages * kWBytes;
   static constexpr int kOffSfw = kOffX + kStages * kXBytes;
   static constexpr int kOffSfx = kOffSfw + kStages * 512;
-  static constexpr int kOffXRaw = kOffSfx + kStages * 512;
-  static constexpr int kOffBar = kOffXRaw + kRawRegion;
-  // full, empty per stage; acc_full, acc_empty x2; drain; epi_sync;
-  // with kQX: raw_full per raw slot
-  static constexpr int kNumBars = 2 * kStages + 2 * 2 + 2 + kMaxRawSlots;
+  static constexpr int kOffBar = kOffSfx + kStages * 512;
+  // full, empty per stage; acc_full, acc_empty x2; drain; epi_sync
+  static constexpr int kNumBars = 2 * kStages + 2 * 2 + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static constexpr int kSfCol0 = 2 * kNM;
   static constexpr int kColsUsed = kSfCol0 + 8 * kStages;
   static constexpr int kTmemCols = kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128 : kColsUsed <= 256 ? 256 : 512;
-  static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kOffXRaw % 1024 == 0, "raw activation region 1024-byte aligned");
+  static_assert(kSmemBytes * kMinBlocksPerSm + 1024 * (kMinBlocksPerSm - 1) <= 232448, "shared memory budget");
 };
 
 __device__ __forceinline__ int64_t dec_unit_start(int b, const DecodeArgs& p) {
@@ -112,9 +112,10 @@ __device__ __forceinline__ void regs_fence_16(uint32_t* r) {
 }
 
 // tmX: the quantized activation (E4M3 [m, k], 128-byte swizzle, box 128 x
-// kNM), or with kQX the bf16 activation [m, k] (no swizzle, box 128 x kNM).
+// kNM); unused with kQX (the activation comes as p.x).
 template <int kNM, int kStages, bool kQX>
-__global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads, 1)
+__global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
+                                  DecodeCfg<kNM, kStages, kQX>::kMinBlocksPerSm)
     gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                         const DecodeArgs p) {
   using Cfg = DecodeCfg<kNM, kStages, kQX>;
@@ -126,7 +127,6 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads, 1)
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint64_t* epi_sync = drain + 1;  // the four epilogue warps meet here (bounded)
-  uint64_t* raw_full = epi_sync + 1;  // kQX: raw activation slab landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 8);
@@ -150,13 +150,12 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads, 1)
     }
     mbar_init(drain, 1);
     mbar_init(epi_sync, 4);
-    for (int j = 0; j < Cfg::kMaxRawSlots; ++j) mbar_init(&raw_full[j], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmW);
-    prefetch_tmap(&tmX);
+    if (!kQX) prefetch_tmap(&tmX);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
@@ -377,88 +376,101 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads, 1)
     }
   } else if (kQX) {
     // ------------------------------------------------------ activation quantizer
-    // Warp qw takes slabs qw, qw + 4, ...; its lane L handles the 16-byte
-    // vector v16 = L % 16 of rows L/16 + 2j < m: K block v16/4, so a block's
-    // four vectors sit in four adjacent lanes of one half-warp and its
-    // maximum is a two-step xor shuffle within that half.
+    // Warp qw takes slabs qw, qw + Q, ... (Q quantizer warps).  Lane L owns the
+    // 32-element K block b = L % 4 of row L/4 < m (m <= 8) of each slab: four
+    // 16-byte loads, the block maximum, one exponent, and 32 E4M3 bytes = two
+    // 16-byte chunks of the swizzled tile row.  The loads of the warp's next
+    // two slabs are in flight while it quantizes the current one.
+    constexpr int Q = Cfg::kQuantWarps;
+    constexpr int kP = 1;
     const int qw = warp - Cfg::kQuantWarp0;
-    const int v16 = lane & 15;
-    const int kblk = v16 >> 2;
-    const unsigned half_mask = (lane & 16) ? 0xFFFF0000u : 0x0000FFFFu;
+    const int b = lane & 3;
+    const int rsub = lane >> 2;
     const int64_t nslabs = u_end - u_begin;
-    const int R = p.raw_slots;  // multiple of 4: slot i % R holds only this warp's slabs
-    const uint32_t raw_bytes = p.raw_bytes;
-    uint8_t* raw_base = smem + Cfg::kOffXRaw;
-    auto slab_kb = [&](int64_t i) { return static_cast<int>((u_begin + i) % p.num_k); };
-    auto load_raw = [&](int64_t i) {
-      const int slot = static_cast<int>(i % R);
-      mbar_arrive_expect_tx(&raw_full[slot], raw_bytes);
-      tma_load_2d(raw_base + slot * raw_bytes, &tmX, &raw_full[slot], slab_kb(i) * 128, 0);
-    };
     // Tile rows m..kNM-1 (and their scale words, with the words of rows
     // kNM..127 that the MMA never reads) are zeroed once; the loop below
     // writes only rows < m.  Word (L, g) of a scale chunk holds row 32g + L.
     const int qt = threadIdx.x - Cfg::kQuantWarp0 * 32;
-    for (int o = qt; o < kStages * (kNM - p.m) * 8; o += 128) {
+    for (int o = qt; o < kStages * (kNM - p.m) * 8; o += 32 * Q) {
       const int st = o / ((kNM - p.m) * 8), rem = o % ((kNM - p.m) * 8);
       reinterpret_cast<uint4*>(smem + Cfg::kOffX + st * Cfg::kXBytes + (p.m + rem / 8) * 128)[rem % 8] =
           make_uint4(0u, 0u, 0u, 0u);
     }
-    for (int w = qt; w < kStages * 128; w += 128) {
+    for (int w = qt; w < kStages * 128; w += 32 * Q) {
       const int L = (w & 127) >> 2, g = w & 3;
       if (32 * g + L >= p.m) reinterpret_cast<uint32_t*>(smem + Cfg::kOffSfx)[(w >> 7) * 128 + L * 4 + g] = 0u;
     }
     // The zeroed rows are read by the tensor core: each thread fences its
-    // stores to the async proxy, and the four warps meet before any of them
-    // arrives on a stage's full barrier.
+    // stores to the async proxy, and the quantizer warps meet before any of
+    // them arrives on a stage's full barrier.
     fence_proxy_async_smem();
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * Q) : "memory");
     griddep_wait();  // the activation may be written by the preceding kernel
-    int64_t issued = qw;  // next slab of this warp to load
-    if (lane == 0)
-      for (; issued < R && issued < nslabs; issued += 4) load_raw(issued);
+    // this lane's block of slab i in each pass (zero past m rows and past k)
+    auto load_slab = [&](int64_t i, uint4 (&v)[kP][4]) {
+      const int64_t col = static_cast<int64_t>((u_begin + i) % p.num_k) * 128 + b * 32;
+#pragma unroll
+      for (int q = 0; q < kP; ++q) {
+        const int r = rsub + 8 * q;
+        const bool in = r < p.m && col < p.k;
+        const __nv_bfloat16* src = p.x + static_cast<int64_t>(r) * p.ldx + col;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) v[q][t] = in ? ld_stream_16(src + 8 * t) : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    uint4 cur[kP][4], nxt[kP][4], nxt2[kP][4];
+    if (qw < nslabs) load_slab(qw, cur);
+    if (qw + Q < nslabs) load_slab(qw + Q, nxt);
     bool ok = true;
-    int64_t i = qw;
-    for (; i < nslabs; i += 4) {
-      const int slot = static_cast<int>(i % R);
+    for (int64_t i = qw; i < nslabs; i += Q) {
+      if (i + 2 * Q < nslabs) load_slab(i + 2 * Q, nxt2);
       const int stage = static_cast<int>(i % kStages);
-      ok = ok && mbar_wait(&raw_full[slot], static_cast<uint32_t>((i / R) & 1), p.timeout_ns, abort_flag,
-                           kSiteQuantRaw);
       ok = ok && mbar_wait(&empty[stage], static_cast<uint32_t>(((i / kStages) & 1) ^ 1), p.timeout_ns, abort_flag,
                            kSiteQuantStage);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
-      const uint8_t* raw = raw_base + slot * raw_bytes;
       uint8_t* xq = smem + Cfg::kOffX + stage * Cfg::kXBytes;
       uint8_t* sfx = smem + Cfg::kOffSfx + stage * 512;
-#pragma unroll 2
-      for (int r = lane >> 4; r < p.m; r += 2) {
-        float f[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(raw + r * 256 + v16 * 16), f);
-        float a = absmax8(f);
-        a = fmaxf(a, __shfl_xor_sync(half_mask, a, 1));
-        a = fmaxf(a, __shfl_xor_sync(half_mask, a, 2));
+#pragma unroll
+      for (int q = 0; q < kP; ++q) {
+        const int r = rsub + 8 * q;
+        if (8 * q >= p.m) break;  // no row of this pass is real
+        // block maximum of |x|: for finite bf16 the magnitude order is the
+        // order of the sign-cleared bit patterns, so a 16-bit unsigned max
+        uint32_t mx = 0;
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          mx = __vmaxu2(__vmaxu2(mx, cur[q][t].x & 0x7FFF7FFFu), __vmaxu2(cur[q][t].y & 0x7FFF7FFFu,
+               __vmaxu2(cur[q][t].z & 0x7FFF7FFFu, cur[q][t].w & 0x7FFF7FFFu)));
+        const float a = __uint_as_float(max(mx & 0xFFFFu, mx >> 16) << 16);
         const int e = mx_exponent(a);
         const float inv = mx_inv_scale(e);
+        uint2 c[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] *= inv;
-        // byte v16*8 of row r: 16-byte chunk v16/2, stored at chunk (v16/2) ^ (r % 8)
-        *reinterpret_cast<uint2*>(xq + r * 128 + (((v16 >> 1) ^ (r & 7)) << 4) + (v16 & 1) * 8) = f32x8_to_e4m3(f);
-        if ((v16 & 3) == 0) sfx[(r & 31) * 16 + ((r & 127) >> 5) * 4 + kblk] = static_cast<uint8_t>(e);
+        for (int t = 0; t < 4; ++t) {
+          float f[8];
+          bf16x8_to_f32(cur[q][t], f);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) f[u] *= inv;
+          c[t] = f32x8_to_e4m3(f);
+        }
+        if (r < p.m) {
+          // bytes 32b..32b+31 of row r: chunks 2b and 2b+1, stored at chunk c ^ (r % 8)
+          uint8_t* row = xq + r * 128;
+          *reinterpret_cast<uint4*>(row + (((2 * b) ^ (r & 7)) << 4)) = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
+          *reinterpret_cast<uint4*>(row + (((2 * b + 1) ^ (r & 7)) << 4)) = make_uint4(c[2].x, c[2].y, c[3].x, c[3].y);
+          sfx[(r & 31) * 16 + ((r & 127) >> 5) * 4 + b] = static_cast<uint8_t>(e);
+        }
       }
       fence_proxy_async_smem();  // the tile and scales are read by the tensor core (async proxy)
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&full[stage]);
-        if (issued < nslabs) {  // the slot's raw data is consumed: load this warp's next slab into it
-          load_raw(issued);
-          issued += 4;
+      if (lane == 0) mbar_arrive(&full[stage]);
+#pragma unroll
+      for (int q = 0; q < kP; ++q)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          cur[q][t] = nxt[q][t];
+          nxt[q][t] = nxt2[q][t];
         }
-      }
-    }
-    // after an early exit, let raw loads still in flight land before the CTA ends
-    if (lane == 0) {
-      for (int64_t j = i; j < issued; j += 4)
-        mbar_wait(&raw_full[j % R], static_cast<uint32_t>((j / R) & 1), p.timeout_ns, nullptr, kSiteQuantDrain);
     }
   }
 

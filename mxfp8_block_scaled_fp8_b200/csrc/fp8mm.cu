@@ -112,23 +112,6 @@ static fp8mm_status make_map(CUtensorMap* map, const void* base, int64_t k, int6
   return FP8MM_OK;
 }
 
-// 2-D map over a row-major bf16 matrix [rows, k] with row stride ld elements,
-// box = 128 elements of K x box_rows rows, no swizzle, zero fill outside.
-static fp8mm_status make_map_bf16(CUtensorMap* map, const void* base, int64_t k, int64_t rows, int64_t ld,
-                                  int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2u};
-  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
-  cuuint32_t es[2] = {1u, 1u};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
-  return FP8MM_OK;
-}
-
 // 3-D map over a library scale buffer viewed as uint32 [n_rt][n_kc][128]
 // (one 512-byte chunk per 128-row tile and 4-block group); box = box_rt chunks
 // of consecutive row tiles at one K group; zero fill past the last row tile.
@@ -183,10 +166,11 @@ using G1 = GemmCfg<false, 256, 4, 2>;
 using G2 = GemmCfg<true, 256, 4, 1>;
 // Small-M ring depth: as many stages as shared memory holds (the weight
 // stream needs ~25 MB in flight GPU-wide to cover the loaded HBM latency).
-constexpr int dec_stages(int nm) { return nm <= 16 ? 11 : nm <= 32 ? 10 : nm <= 48 ? 9 : 8; }
-// With the activation quantized in the kernel (m <= 16), its raw slabs take
-// shared memory too.
-constexpr int dec_stages_qx(int nm) { return nm <= 16 ? 10 : 0; }
+// Stages of the small-M kernel: token tiles up to 32 run two CTAs per SM
+// (half the shared memory each), larger ones one CTA with a deeper ring.
+constexpr int dec_stages(int nm) { return nm <= 16 ? 5 : nm <= 32 ? 5 : nm <= 48 ? 9 : 8; }
+// With the activation quantized in the kernel (m <= 8).
+constexpr int dec_stages_qx(int nm) { return nm <= 16 ? 5 : 0; }
 
 __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
   __shared__ uint64_t bar;
@@ -409,13 +393,11 @@ static fp8mm_status launch_small_m(const void* a, const uint8_t* sfa, const void
   CUtensorMap tw, tx;
   fp8mm_status st = make_map(&tw, b, k, n, 128);
   if (st != FP8MM_OK) return st;
-  st = qx ? make_map_bf16(&tx, a, k, m, lda, static_cast<int>(m)) : make_map(&tx, a, k, m, nm);
-  if (st != FP8MM_OK) return st;
-  if (qx) {  // m <= 16: raw activation slabs of m rows x 128 bf16, a multiple of 4 slots
-    constexpr int kRegion = DecodeCfg<16, dec_stages_qx(16), true>::kRawRegion;
-    p.raw_bytes = static_cast<uint32_t>(m) * 256u;
-    p.raw_slots = static_cast<int>(std::min<int64_t>(16, kRegion / p.raw_bytes)) & ~3;
-    return launch_small_m_t<16, true>(tw, tx, p, stream, dev.device);
+  if (!qx && (st = make_map(&tx, a, k, m, nm)) != FP8MM_OK) return st;
+  if (qx) {  // m <= 8: the activation is read by the kernel itself
+    p.x = static_cast<const __nv_bfloat16*>(a);
+    p.ldx = lda;
+    return launch_small_m_t<16, true>(tw, tw, p, stream, dev.device);
   }
   switch (nm) {
     case 16: return launch_small_m_t<16>(tw, tx, p, stream, dev.device);
@@ -613,7 +595,7 @@ fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e
 // Largest m whose activation is quantized inside the small-M kernel; above it
 // the per-CTA re-quantization of every K slab costs more than a separate
 // quantizer launch, which then writes into the workspace.
-constexpr int64_t kQuantInKernelMaxM = 16;
+constexpr int64_t kQuantInKernelMaxM = 8;
 
 static size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 

@@ -20,8 +20,7 @@ enum DevErr : unsigned { kDevErrTimeout = 1 };
 
 enum WaitSite : unsigned {
   kSiteProducerEmpty = 1, kSiteMmaFull = 2, kSiteMmaAccEmpty = 3, kSiteEpiAccFull = 4,
-  kSiteDrain = 5, kSiteProducerDrain = 6, kSiteSelfTest = 7, kSiteEpiSync = 8, kSiteQuantRaw = 9,
-  kSiteQuantStage = 10, kSiteQuantDrain = 11,
+  kSiteDrain = 5, kSiteProducerDrain = 6, kSiteSelfTest = 7, kSiteEpiSync = 8, kSiteQuantStage = 9,
 };
 
 __device__ __forceinline__ void record_error(unsigned kind, unsigned site) {

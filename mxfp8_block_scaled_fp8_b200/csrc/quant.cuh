@@ -23,9 +23,13 @@
 
 namespace fp8mm {
 
+// 16-byte streaming load (not kept in L1).  Coherent (no .nc): the kernels
+// read inputs that the preceding kernel, overlapping them through
+// programmatic dependent launch, may still be writing before their
+// griddepcontrol.wait.
 __device__ __forceinline__ uint4 ld_stream_16(const void* p) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;

@@ -216,8 +216,8 @@ def mxfp8_quantize_gemm(a: torch.Tensor, b: torch.Tensor, sf_b: torch.Tensor, c:
                         workspace: torch.Tensor | None = None, kernel: int = KERNEL_AUTO, small_m_ctas: int = 0,
                         weights_ready: bool = False, stream=None) -> torch.Tensor:
     """C bf16 [m, n] = mxfp8_gemm(mxfp8_quantize(a), b) for m <= 64 from the bf16 activation a [m, k]:
-    quantized inside the GEMM kernel for m <= 16, else by its own launch into the workspace tail
-    (workspace of quantize_gemm_workspace_bytes(m, n, k, small_m_ctas) bytes, required for m > 16)."""
+    quantized inside the GEMM kernel for m <= 8, else by its own launch into the workspace tail
+    (workspace of quantize_gemm_workspace_bytes(m, n, k, small_m_ctas) bytes, required for m > 8)."""
     b = _u8(b)
     _need(a, torch.bfloat16, "a"); _need(b, torch.uint8, "b"); _need(sf_b, torch.uint8, "sf_b")
     m, k = a.shape

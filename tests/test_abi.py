@@ -70,7 +70,7 @@ def test_argument_errors_without_a_gpu():
     tiled = binding.Opts(None, 0, binding.KERNEL_TILED, 0, 0)
     assert Q(P(fake), 64, P(fake), P(fake), 4, 4, 64, P(fake), 8, ctypes.byref(tiled), None) == 2
     assert Q(None, 64, None, None, 0, 4, 64, None, 8, None, None) == 0                 # m == 0
-    assert Q(P(fake), 64, P(fake), P(fake), 32, 4, 64, P(fake), 8, None, None) == 6     # m > 16 needs a workspace
+    assert Q(P(fake), 64, P(fake), P(fake), 9, 4, 64, P(fake), 8, None, None) == 6      # m > 8 needs a workspace
     # empty problems are no-ops and need no device
     assert L.fp8_gemm(None, None, 0, 4, 16, None, None, None, 8, None, None) == 0
     assert L.mxfp8_quantize(None, 0, 64, 64, None, 64, None, None) == 0
@@ -83,8 +83,8 @@ def test_workspace_sizes():
     assert fp8mm.workspace_bytes(1, 4096, 14336, 148) == 2 * 148 * 128 * 16 * 4 + 256
     assert fp8mm.workspace_bytes(65, 4096, 4096, 148) == 0            # only for m <= 64
     assert fp8mm.workspace_bytes(8, 128, 128, 148) == 2 * 1 * 128 * 16 * 4 + 256   # clamped to 1 unit
-    # activation-quantizing GEMM: the same for m <= 16, plus the quantized activation and scales above
-    assert fp8mm.quantize_gemm_workspace_bytes(16, 14336, 4096, 148) == fp8mm.workspace_bytes(16, 14336, 4096, 148)
+    # activation-quantizing GEMM: the same for m <= 8, plus the quantized activation and scales above
+    assert fp8mm.quantize_gemm_workspace_bytes(8, 14336, 4096, 148) == fp8mm.workspace_bytes(8, 14336, 4096, 148)
     assert (fp8mm.quantize_gemm_workspace_bytes(33, 4096, 14336, 148) ==
             fp8mm.workspace_bytes(33, 4096, 14336, 148) + 33 * 14336 + fp8mm.sf_bytes(33, 14336))
     assert fp8mm.quantize_gemm_workspace_bytes(65, 4096, 4096, 148) == 0

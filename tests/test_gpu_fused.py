@@ -68,7 +68,8 @@ def test_fused_decode_sweep(weights, name, m):
     assert torch.equal(c, c2), "second call with the same workspace differs"
 
 
-@pytest.mark.parametrize("m,n,k", [(1, 1, 32), (3, 200, 96), (9, 260, 4128), (16, 129, 8192), (17, 130, 4128),
+@pytest.mark.parametrize("m,n,k", [(1, 1, 32), (3, 200, 96), (8, 260, 4128), (9, 300, 4096), (16, 129, 8192),
+                                   (17, 130, 4128),
                                    (33, 1000, 64), (49, 300, 160), (64, 384, 320)])
 def test_fused_ragged_strided(m, n, k):
     """Ragged m, n and k (k a multiple of 32, not of 128), a row stride wider
@@ -89,7 +90,7 @@ def test_fused_ragged_strided(m, n, k):
         torch.cuda.synchronize()
         gu.check_gemm(c, c_ref, bound, f"fused ragged {m}x{n}x{k} ctas={ctas}")
         assert torch.equal(c, c_un), f"fused ragged {m}x{n}x{k} ctas={ctas} differs from quantize + GEMM"
-    if m <= 16:                                                 # no workspace: one CTA per tile
+    if m <= 8:                                                  # no workspace: one CTA per tile
         c = fp8mm.mxfp8_quantize_gemm(xd, gw, gsfw)
         torch.cuda.synchronize()
         gu.check_gemm(c, c_ref, bound, f"fused ragged {m}x{n}x{k} one CTA per tile")
@@ -173,6 +174,6 @@ def test_fused_degenerate_and_errors(weights):
         fp8mm.mxfp8_quantize_gemm(x[:8], gw, gsfw, workspace=torch.zeros(256, dtype=torch.uint8, device="cuda"))
     with pytest.raises(fp8mm.Fp8mmError):
         fp8mm.mxfp8_quantize_gemm(x[:8], gw, gsfw, kernel=fp8mm.KERNEL_TILED)
-    with pytest.raises(fp8mm.Fp8mmError):                          # m > 16 without room for the activation
-        fp8mm.mxfp8_quantize_gemm(x[:32], gw, gsfw, workspace=_ws(32, n, k))
+    with pytest.raises(fp8mm.Fp8mmError):                          # m > 8 without room for the activation
+        fp8mm.mxfp8_quantize_gemm(x[:9], gw, gsfw, workspace=_ws(9, n, k))
     assert fp8mm.last_device_error() == 0
