@@ -395,7 +395,7 @@ def run_ours(args):
                 "ms_per_step": e2e_ms},
         "gpu_launches": 2 * args.steps,
         "kernels": {"mxfp8_quantize_ms": q_ms, "mxfp8_gemm_ms": g_ms},
-        "roofline": {"bound": "tensor", "kernel": "gemm_tiled_kernel<mx> (mxfp8_gemm)", "achieved": achieved,
+        "roofline": {"bound": "tensor", "kernel": "gemm_pair_kernel<mx> (mxfp8_gemm, 256x256 tiles on 2-CTA clusters)", "achieved": achieved,
                      "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
                      "traffic": _ncu_traffic("mxfp8_gemm_ffn_up"),
                      "peak_note": f"FP8 dense = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s "
