@@ -530,7 +530,9 @@ fp8mm_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
   if (st != FP8MM_OK) return st;
   const int64_t n_kc = cdiv(k, 128);
   const int64_t rows_pad = cdiv(rows, 128) * 128;
-  const int grid = static_cast<int>(std::min<int64_t>(rows_pad, static_cast<int64_t>(dev.sms) * 8));
+  // one warp per 32-block segment of a padded row, 8 warps per CTA
+  const int64_t segments = rows_pad * cdiv(cdiv(k, 128) * 4, 32);
+  const int grid = static_cast<int>(std::min<int64_t>(cdiv(segments, kQ2Threads / 32), static_cast<int64_t>(dev.sms) * 8));
   st = launch_pdl(quant_mx_kernel, dim3(grid), dim3(kQ2Threads), 0, static_cast<cudaStream_t>(stream),
                   static_cast<const __nv_bfloat16*>(x_bf16), rows, k, ld_x, static_cast<uint8_t*>(q_e4m3), ld_q, sf,
                   static_cast<int>(n_kc), rows_pad);

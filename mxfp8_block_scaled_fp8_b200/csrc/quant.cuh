@@ -9,8 +9,8 @@
 //   "[sglang] FlashInfer v0.6.7 MXFP8 Gemm 통합", section 1 (one uint8 scale
 //   per 32 elements).
 //
-// Both kernels read bf16 with 16-byte vector loads and write E4M3 with
-// 8-byte stores; a warp always covers a contiguous run of one row.  They are
+// Both kernels read bf16 with 16-byte vector loads; a warp always covers a
+// contiguous run of one row.  They are
 // launched with programmatic dependent launch and wait for the preceding
 // kernel before touching memory, so only their launch overlaps it.
 #pragma once
@@ -216,69 +216,97 @@ __device__ __forceinline__ float mx_inv_scale(int e) {
   return (e < 254) ? __uint_as_float(static_cast<uint32_t>(254 - e) << 23) : __uint_as_float(0x00400000u);
 }
 
-constexpr int kQ2Threads = 256;   // 8 warps = 16 groups of 128 elements per pass
-constexpr int kQ2Passes = 8;      // passes whose loads are in flight together
+constexpr int kQ2Threads = 256;
 
-// One CTA per row of the padded scale buffer (grid-stride).  A "group" is one
-// row x 4 consecutive K-blocks = 128 elements = 16 lanes x 16 bytes and
-// produces one 32-bit word of the scale layout; a warp handles two groups per
-// pass and the CTA 16.  All loads of up to kQ2Passes passes are issued before
-// any arithmetic.  Rows >= rows and blocks >= k/32 (padding) get exponent 0.
+// Exact maximum of |x| over the 32 bf16 values of four 16-byte vectors, as
+// fp32: for finite bf16 the order of magnitudes is the order of the
+// sign-cleared bit patterns, so it is a 16-bit unsigned maximum.
+__device__ __forceinline__ float bf16x32_absmax(const uint4 (&v)[4]) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int t = 0; t < 4; ++t)
+    m = __vmaxu2(__vmaxu2(m, v[t].x & 0x7FFF7FFFu),
+                 __vmaxu2(v[t].y & 0x7FFF7FFFu, __vmaxu2(v[t].z & 0x7FFF7FFFu, v[t].w & 0x7FFF7FFFu)));
+  return __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
+}
+
+// One warp per segment of 32 consecutive K blocks (1024 elements) of one
+// padded row, grid-stride over the rows_pad x ceil(n_kc*4 / 32) segments;
+// lane L owns block kb = 32*seg + L: four 16-byte loads, its maximum, the
+// exponent, 32 E4M3 bytes, and the lanes L % 4 == 0 gather the four
+// exponents of one scale word.  The next segment's loads are in flight
+// while the current one is converted.  Rows >= rows and blocks >= k/32
+// (padding) get exponent 0 and no codes.
 __global__ void __launch_bounds__(kQ2Threads) quant_mx_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
                                                               int64_t k, int64_t ld_x, uint8_t* __restrict__ q,
                                                               int64_t ld_q, uint8_t* __restrict__ sf, int n_kc,
                                                               int64_t rows_pad) {
   const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int half = lane >> 4;        // which of the warp's two groups
-  const int sub = lane & 15;         // lane within the group
-  const int kb_in = sub >> 2;        // K-block within the group
-  const int v_in = sub & 3;          // 16-byte vector within the block
-  const int gid = warp * 2 + half;   // group within a pass
   const int nkb = static_cast<int>(k / 32);
-  griddep_launch_dependents();       // a following GEMM may start prefetching its weights
-  griddep_wait();                    // x and the outputs may belong to the preceding kernel
-  for (int64_t row = blockIdx.x; row < rows_pad; row += gridDim.x) {
-    const bool row_real = row < rows;
-    const __nv_bfloat16* xr = x + (row_real ? row : 0) * ld_x;
-    uint8_t* qr = q + (row_real ? row : 0) * ld_q;
-    uint8_t* sf_row = sf + (row / 128) * static_cast<int64_t>(n_kc) * 512 + (row % 32) * 16 + ((row % 128) / 32) * 4;
-    for (int kc0 = 0; kc0 < n_kc; kc0 += 16 * kQ2Passes) {
-      uint4 v[kQ2Passes];
+  const int nkb4 = n_kc * 4;
+  const int segs = (nkb4 + 31) / 32;
+  const int64_t total = rows_pad * segs;
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * (kQ2Threads / 32);
+  int64_t w = static_cast<int64_t>(blockIdx.x) * (kQ2Threads / 32) + (threadIdx.x >> 5);
+  // (row, seg) of w, advanced without division
+  int64_t row = w / segs;
+  int seg = static_cast<int>(w - row * segs);
+  const int64_t drow = wstride / segs;
+  const int dseg = static_cast<int>(wstride - drow * segs);
+  const bool q16 = (reinterpret_cast<uintptr_t>(q) % 16 == 0) && (ld_q % 16 == 0);
+  griddep_launch_dependents();  // a following GEMM may start prefetching its weights
+  griddep_wait();               // x and the outputs may belong to the preceding kernel
+  auto load = [&](int64_t r, int sg, uint4 (&v)[4]) {
+    const int kb = sg * 32 + lane;
+    const bool real = r < rows && kb < nkb;
+    const __nv_bfloat16* src = x + (real ? r : 0) * ld_x + static_cast<int64_t>(kb) * 32;
 #pragma unroll
-      for (int ps = 0; ps < kQ2Passes; ++ps) {
-        const int kc = kc0 + ps * 16 + gid;
-        const int kb = kc * 4 + kb_in;
-        v[ps] = (row_real && kc < n_kc && kb < nkb) ? ld_stream_16(xr + kb * 32 + v_in * 8) : make_uint4(0, 0, 0, 0);
-      }
+    for (int t = 0; t < 4; ++t) v[t] = real ? ld_stream_16(src + 8 * t) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  uint4 cur[4], nxt[4];
+  if (w < total) load(row, seg, cur);
+  for (; w < total; w += wstride) {
+    int64_t nrow = row + drow;
+    int nseg = seg + dseg;
+    if (nseg >= segs) {
+      nseg -= segs;
+      ++nrow;
+    }
+    if (w + wstride < total) load(nrow, nseg, nxt);
+    const int kb = seg * 32 + lane;
+    const bool real = row < rows && kb < nkb;
+    const int e = real ? mx_exponent(bf16x32_absmax(cur)) : 0;
+    if (real) {
+      const float inv = mx_inv_scale(e);  // exact: power-of-two scaling
+      uint2 c[4];
 #pragma unroll
-      for (int ps = 0; ps < kQ2Passes; ++ps) {
-        if (kc0 + ps * 16 >= n_kc) break;  // the same for every thread of the CTA
-        const int kc = kc0 + ps * 16 + gid;
-        const int kb = kc * 4 + kb_in;
-        const bool real = row_real && kc < n_kc && kb < nkb;
+      for (int t = 0; t < 4; ++t) {
         float f[8];
-        bf16x8_to_f32(v[ps], f);
-        float amax = absmax8(f);
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-        const int e = real ? mx_exponent(amax) : 0;
-        if (real) {
-          const float inv = mx_inv_scale(e);
+        bf16x8_to_f32(cur[t], f);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) f[j] *= inv;  // exact: power-of-two scaling
-          *reinterpret_cast<uint2*>(qr + kb * 32 + v_in * 8) = f32x8_to_e4m3(f);
-        }
-        // gather the group's four exponents into its first lane
-        const int base = half * 16;
-        const uint32_t e0 = __shfl_sync(0xFFFFFFFFu, e, base + 0);
-        const uint32_t e1 = __shfl_sync(0xFFFFFFFFu, e, base + 4);
-        const uint32_t e2 = __shfl_sync(0xFFFFFFFFu, e, base + 8);
-        const uint32_t e3 = __shfl_sync(0xFFFFFFFFu, e, base + 12);
-        if (sub == 0 && kc < n_kc)
-          *reinterpret_cast<uint32_t*>(sf_row + static_cast<int64_t>(kc) * 512) = e0 | (e1 << 8) | (e2 << 16) | (e3 << 24);
+        for (int u = 0; u < 8; ++u) f[u] *= inv;
+        c[t] = f32x8_to_e4m3(f);
+      }
+      uint8_t* dst = q + row * ld_q + static_cast<int64_t>(kb) * 32;
+      if (q16) {
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
+        reinterpret_cast<uint4*>(dst)[1] = make_uint4(c[2].x, c[2].y, c[3].x, c[3].y);
+      } else {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) reinterpret_cast<uint2*>(dst)[t] = c[t];
       }
     }
+    // scale word of blocks kb..kb+3 (lanes L..L+3, L % 4 == 0)
+    const uint32_t e1 = __shfl_down_sync(0xFFFFFFFFu, static_cast<uint32_t>(e), 1);
+    const uint32_t e2 = __shfl_down_sync(0xFFFFFFFFu, static_cast<uint32_t>(e), 2);
+    const uint32_t e3 = __shfl_down_sync(0xFFFFFFFFu, static_cast<uint32_t>(e), 3);
+    if ((lane & 3) == 0 && kb < nkb4)
+      *reinterpret_cast<uint32_t*>(sf + ((row / 128) * n_kc + kb / 4) * 512 + (row % 32) * 16 + ((row % 128) / 32) * 4) =
+          static_cast<uint32_t>(e) | (e1 << 8) | (e2 << 16) | (e3 << 24);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) cur[t] = nxt[t];
+    row = nrow;
+    seg = nseg;
   }
 }
 
