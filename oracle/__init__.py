@@ -38,6 +38,10 @@ def lib():
         L.orc_mx_exponent.restype = ctypes.c_int
         L.orc_quantize_rowwise.argtypes = [P, I64, I64, I64, P, I64, P, ctypes.c_int]
         L.orc_quantize_rowwise.restype = None
+        L.orc_tensor_scale.argtypes = [P, I64, I64, I64]
+        L.orc_tensor_scale.restype = ctypes.c_float
+        L.orc_quantize_static.argtypes = [P, I64, I64, I64, ctypes.c_float, P, I64, ctypes.c_int]
+        L.orc_quantize_static.restype = None
         L.orc_mx_quantize.argtypes = [P, I64, I64, I64, P, I64, P, ctypes.c_int]
         L.orc_mx_quantize.restype = None
         L.orc_gemm_rowwise.argtypes = [P, P, I64, I64, I64, P, P, P, P, ctypes.c_int]
@@ -88,6 +92,34 @@ def quantize_rowwise(x_bits: np.ndarray, nthreads: int = 0):
     lib().orc_quantize_rowwise(_ptr(x), R, K, K, _ptr(q), K, _ptr(s),
                                nthreads or default_threads())
     return q, s
+
+
+def tensor_scale(x_bits: np.ndarray) -> np.float32:
+    """Per-tensor scale fp32(max|x| / 448) (1 for an all-zero tensor)."""
+    x = _c(x_bits, np.uint16)
+    rows, k = x.shape
+    return np.float32(lib().orc_tensor_scale(_ptr(x), rows, k, k))
+
+
+def quantize_static(x_bits: np.ndarray, scale, nthreads: int = 0) -> np.ndarray:
+    """E4M3 codes of fp32(x / scale) for one given fp32 scale."""
+    x = _c(x_bits, np.uint16)
+    rows, k = x.shape
+    q = np.empty((rows, k), dtype=np.uint8)
+    lib().orc_quantize_static(_ptr(x), rows, k, k, ctypes.c_float(float(np.float32(scale))), _ptr(q), k,
+                              nthreads or default_threads())
+    return q
+
+
+def concat_mla_k(k_nope: np.ndarray, k_rope: np.ndarray) -> np.ndarray:
+    """Key assembly of page "[flashinfer] FlashInfer, FP8 지원으로 장문 컨텍스트 추론
+    성능을 극적으로 향상시키다" (코드 분석 items 1 and 3): for every token t and head h,
+    the nope part of the key followed by its rope part; a k_rope with one head is the
+    same rope vector for every head.  Inputs [T, H, nope] and [T, H or 1, rope] of any
+    element type; the output [T, H, nope + rope] holds the input elements unchanged."""
+    T, H, _ = k_nope.shape
+    rope = np.broadcast_to(k_rope, (T, H, k_rope.shape[2]))
+    return np.concatenate([k_nope, rope], axis=2)
 
 
 def mx_quantize(x_bits: np.ndarray, nthreads: int = 0):

@@ -120,6 +120,32 @@ void orc_quantize_rowwise(const uint16_t* x, int64_t rows, int64_t k, int64_t ld
     parallel_rows(rows, nthreads, rowwise_row, &c);
 }
 
+float orc_tensor_scale(const uint16_t* x, int64_t rows, int64_t k, int64_t ld_x) {
+    float amax = 0.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < k; ++j) {
+            float a = fabsf(bf16_to_float(x[r * ld_x + j]));
+            if (a > amax) amax = a;
+        }
+    return (amax == 0.0f) ? 1.0f : (float)((double)amax / 448.0);
+}
+
+typedef struct { const uint16_t* x; int64_t k, ld_x; float s; uint8_t* q; int64_t ld_q; } static_ctx;
+
+static void static_row(void* p, int64_t r) {
+    static_ctx* c = (static_ctx*)p;
+    for (int64_t j = 0; j < c->k; ++j) {
+        float v = bf16_to_float(c->x[r * c->ld_x + j]) / c->s;   /* fp32 quotient, IEEE RN */
+        c->q[r * c->ld_q + j] = orc_e4m3_encode((double)v);
+    }
+}
+
+void orc_quantize_static(const uint16_t* x, int64_t rows, int64_t k, int64_t ld_x, float s,
+                         uint8_t* q, int64_t ld_q, int nthreads) {
+    static_ctx c = {x, k, ld_x, s, q, ld_q};
+    parallel_rows(rows, nthreads, static_row, &c);
+}
+
 static void mx_row(void* p, int64_t r) {
     quant_ctx* c = (quant_ctx*)p;
     const uint16_t* xr = c->x + r * c->ld_x;

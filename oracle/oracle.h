@@ -52,6 +52,17 @@ uint8_t orc_e4m3_encode(double v);
  * i.e. the amax/448 rule of [DG] listing 3 restricted to UE8M0 scales ([MX]). */
 int orc_mx_exponent(double amax);
 
+/* Per-tensor scale ([DG] listing 3, _calibrate_scales as printed: one scale
+ * per tensor, max |x| over all of it / 448): s = fp32(amax / 448), 1 when the
+ * tensor is all zero.  x: bf16 bit patterns, rows x k, row stride ld_x. */
+float orc_tensor_scale(const uint16_t* x, int64_t rows, int64_t k, int64_t ld_x);
+
+/* Static-scale quantizer: q[r, j] = encode(fp32(x[r, j] / s)) with one given
+ * fp32 scale s > 0 for the whole tensor (a calibrated per-tensor scale, as
+ * [DG] listing 3 computes once and then uses for inference). */
+void orc_quantize_static(const uint16_t* x, int64_t rows, int64_t k, int64_t ld_x, float s,
+                         uint8_t* q, int64_t ld_q, int nthreads);
+
 /* Per-row quantizer (mode 1).  For each row r of x (bf16 bit patterns,
  * row stride ld_x elements): amax = max |x|; s[r] = fp32(amax / 448)
  * (s = 1 when amax == 0); q[r, j] = encode(fp32(x[r, j] / s[r])).
