@@ -221,6 +221,51 @@ def _rows_measurements(fp8mm, synthetic, peaks, only=None):
             out["fp8_gemm_8192x2048x8192"] = {"ms": t, "TFLOPS": tf, "frac_fp8_peak": tf / fp8_peak}
         del a, bt
 
+    if want("tensor_scale_8192x8192") or want("quantize_static_8192x8192") or want("fp8_gemm_e4m3_out_8192x2048x8192"):
+        # per-tensor calibration scale, static-scale quantizer, GEMM with E4M3 output
+        a, bt = synthetic.attn()
+        a, bt = a.to(dev), bt.to(dev)
+        R, Kq = a.shape
+        xs = [a] + [a.clone() for _ in range(_copies(a.numel() * 2) - 1)]
+        s_dev = torch.empty(1, dtype=torch.float32, device=dev)
+        if want("tensor_scale_8192x8192"):
+            t = _graph_time([lambda x=x: fp8mm.fp8_tensor_scale(x, s_dev) for x in xs])
+            gbs = 2.0 * R * Kq / (t * 1e-3) / 1e9
+            out["tensor_scale_8192x8192"] = {"ms": t, "GB/s": gbs, "frac_hbm": gbs / hbm}
+        fp8mm.fp8_tensor_scale(a, s_dev)
+        qa = torch.empty(a.shape, dtype=torch.uint8, device=dev)
+        if want("quantize_static_8192x8192"):
+            t = _graph_time([lambda x=x: fp8mm.fp8_quantize_static(x, s_dev, qa) for x in xs])
+            gbs = 3.0 * R * Kq / (t * 1e-3) / 1e9
+            out["quantize_static_8192x8192"] = {"ms": t, "GB/s": gbs, "frac_hbm": gbs / hbm}
+        del xs
+        if want("fp8_gemm_e4m3_out_8192x2048x8192"):
+            qa, sa = fp8mm.fp8_quantize_rowwise(a)
+            qb, sb = fp8mm.fp8_quantize_rowwise(bt)
+            c8 = torch.empty((R, bt.shape[0]), dtype=torch.uint8, device=dev)
+            so = torch.ones(1, dtype=torch.float32, device=dev)
+            t = _graph_time([lambda: fp8mm.fp8_gemm_e4m3_out(qa, qb, sa, sb, so, c8)] * 4)
+            tf = 2.0 * 8192 * 2048 * 8192 / (t * 1e-3) / 1e12
+            out["fp8_gemm_e4m3_out_8192x2048x8192"] = {"ms": t, "TFLOPS": tf, "frac_fp8_peak": tf / fp8_peak}
+        del a, bt
+
+    if want("concat_mla_k_16384x128"):
+        # MLA key assembly in FP8: 16384 tokens x 128 heads, nope 128 + rope 64 (one per token)
+        T, H = 16384, 128
+        g = torch.Generator(device=dev).manual_seed(5)
+        sets = []
+        per = T * H * 128 + T * 64
+        for _ in range(_copies(per)):
+            nope = torch.randint(0, 256, (T, H, 128), device=dev, dtype=torch.uint8, generator=g)
+            rope = torch.randint(0, 256, (T, 1, 64), device=dev, dtype=torch.uint8, generator=g)
+            sets.append((nope.view(torch.float8_e4m3fn), rope.view(torch.float8_e4m3fn)))
+        kout = torch.empty((T, H, 192), dtype=torch.float8_e4m3fn, device=dev)
+        t = _graph_time([lambda n_=n_, r_=r_: fp8mm.concat_mla_k(n_, r_, kout) for n_, r_ in sets])
+        byts = T * H * 128 + T * 64 + T * H * 192
+        out["concat_mla_k_16384x128"] = {"ms": t, "GB/s": byts / (t * 1e-3) / 1e9,
+                                         "frac_hbm": byts / (t * 1e-3) / 1e9 / hbm}
+        del sets, kout
+
     if want("mxfp8_gemm_2048x1024x4096"):
         # Q.K^T shape: 64 output tiles, fewer than the 148 SMs
         a, bt = synthetic.qk()

@@ -127,6 +127,38 @@ fp8mm_status fp8_gemm(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t
                       const float* scale_a, const float* scale_b, void* c_bf16, int64_t ldc,
                       const fp8mm_opts* opt, void* stream);
 
+/* ------------------------------------------------ per-tensor scale, FP8 out */
+
+/* Per-tensor scale -- page "FP8 推理基础设施（五）：从 DeepGEMM 到 vLLM",
+ * listing 3 (_calibrate_scales as printed: one scale per tensor):
+ *   *scale = fp32(max |x| / 448) over the whole [rows, k] bf16 tensor (row
+ *   stride ld_x elements), 1.0 for an all-zero tensor.
+ * *scale is a device fp32 that the call overwrites (it is also the work word
+ * of the reduction).  Requires k % 8 == 0, x 16-byte aligned, ld_x % 8 == 0,
+ * rows * k / 8 < 2^32.  Three stream operations: a 4-byte memset and two
+ * kernels.  rows == 0 or k == 0 writes 1.0. */
+fp8mm_status fp8_tensor_scale(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, float* scale,
+                              void* stream);
+
+/* Static-scale quantizer (a calibrated per-tensor scale, as the same listing
+ * uses it at inference; also the FP8 KV-cache quantizer):
+ *   q[r, j] = E4M3_RNE_sat(fp32(x[r, j] / *scale))   (IEEE fp32 quotient)
+ * scale: device fp32 > 0, read once by the kernel.  Layout and alignment
+ * rules as fp8_quantize_rowwise; rows * k / 8 < 2^32. */
+fp8mm_status fp8_quantize_static(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, const float* scale,
+                                 void* q_e4m3, int64_t ld_q, void* stream);
+
+/* fp8_gemm with an E4M3 output (listing 1's C_fp8), scaled for the next
+ * layer:  c[m, n] = E4M3_RNE_sat( fp32(scale_a[m] scale_b[n] acc[m, n]) / *scale_out )
+ * where acc is the fp32 tensor-core sum over K; scale_out is a device fp32
+ * (e.g. from fp8_tensor_scale on calibration data).  c_e4m3 [m, n] bytes with
+ * row stride ldc >= n, any alignment; other arguments and rules as fp8_gemm.
+ * The quotient is within one fp32 step of the IEEE quotient (exact tensor-
+ * core accumulation order is not defined anyway); outputs past +-448 saturate. */
+fp8mm_status fp8_gemm_e4m3_out(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t n, int64_t k,
+                               const float* scale_a, const float* scale_b, const float* scale_out, void* c_e4m3,
+                               int64_t ldc, const fp8mm_opts* opt, void* stream);
+
 /* ---------------------------------------------------------------- mode 2 */
 
 /* Scale-factor (SF) layout of this library.  Rows are padded to a multiple of
@@ -205,6 +237,25 @@ size_t fp8mm_quantize_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k, int3
 /* Workspace bytes the small-M kernel needs for this shape with `ctas` CTAs
  * (0 = one per SM of the current device; on a host without a GPU, 148). */
 size_t fp8mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas);
+
+/* ---------------------------------------------------------------- KV cache */
+
+/* Key assembly for multi-head latent attention, for FP8 (E4M3 / E5M2) or
+ * 16-bit elements -- page "[flashinfer] FlashInfer, FP8 지원으로 장문 컨텍스트
+ * 추론 성능을 극적으로 향상시키다", 코드 분석 items 1 and 3:
+ *   k_out[t, h, 0:nope_dim]                   = k_nope[t, h, :]
+ *   k_out[t, h, nope_dim:nope_dim + rope_dim] = k_rope[t, h, :]
+ * for t < num_tokens, h < num_heads.  A copy: the output bytes are the input
+ * bytes.  rope_stride_h = 0 broadcasts one rope vector per token to every
+ * head.  All strides are in elements of elem_bytes (1 or 2) bytes; every
+ * pointer is 16-byte aligned and every stride, nope_dim and rope_dim times
+ * elem_bytes is a multiple of 16 (FP8MM_ERR_ALIGN otherwise);
+ * num_tokens * num_heads * (nope_dim + rope_dim) * elem_bytes / 16 < 2^32.
+ * num_tokens == 0 or num_heads == 0 is a no-op. */
+fp8mm_status concat_mla_k(const void* k_nope, const void* k_rope, void* k_out, int64_t num_tokens,
+                          int64_t num_heads, int64_t nope_dim, int64_t rope_dim, int64_t elem_bytes,
+                          int64_t nope_stride_t, int64_t nope_stride_h, int64_t rope_stride_t,
+                          int64_t rope_stride_h, int64_t out_stride_t, int64_t out_stride_h, void* stream);
 
 /* ---------------------------------------------------------------- misc */
 

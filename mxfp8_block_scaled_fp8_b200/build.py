@@ -12,7 +12,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OUT = os.path.join(PKG, "libfp8mm.so")
 SOURCES = ["fp8mm.cu"]
-HEADERS = ["ptx.cuh", "quant.cuh", "gemm.cuh", "gemm2.cuh", "decode.cuh"]
+HEADERS = ["ptx.cuh", "quant.cuh", "gemm.cuh", "gemm2.cuh", "decode.cuh", "kvcache.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -9,11 +9,13 @@
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <set>
 #include <utility>
 
 #include "decode.cuh"
+#include "kvcache.cuh"
 #include "gemm.cuh"
 #include "gemm2.cuh"
 #include "ptx.cuh"
@@ -186,9 +188,11 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
 }
 
 // ------------------------------------------------------------------ launchers
+// c8 != nullptr (mode 1 only): E4M3 output c8 = E4M3(C / *s_out) instead of bf16 c.
 static fp8mm_status launch_tiled(bool mx, const void* a, const void* b, const uint8_t* sfa, const uint8_t* sfb,
                                  int64_t m, int64_t n, int64_t k, const float* sa, const float* sb, void* c,
-                                 int64_t ldc, cudaStream_t stream, const DeviceInfo& dev) {
+                                 int64_t ldc, cudaStream_t stream, const DeviceInfo& dev, uint8_t* c8 = nullptr,
+                                 const float* s_out = nullptr) {
   CUtensorMap ta, tb;
   fp8mm_status st = make_map(&ta, a, k, m, kBM);
   if (st != FP8MM_OK) return st;
@@ -211,8 +215,14 @@ static fp8mm_status launch_tiled(bool mx, const void* a, const void* b, const ui
   p.n_kc = static_cast<int>(cdiv(k, 128));
   p.sfb_row_tiles = static_cast<int>(cdiv(n, 128));
   p.timeout_ns = wait_timeout_ns();
+  p.c8 = c8;
+  p.s_out = s_out;
   const int grid = std::min(p.num_tiles, dev.sms);
-  if (mx) {
+  if (c8 != nullptr) {
+    auto kern = gemm_tiled_kernel<false, 256, 4, 2, true>;
+    if ((st = ensure_smem(reinterpret_cast<const void*>(kern), G1::kSmemBytes, dev.device)) != FP8MM_OK) return st;
+    kern<<<grid, kGemmThreads, G1::kSmemBytes, stream>>>(ta, tb, p);
+  } else if (mx) {
     auto kern = gemm_tiled_kernel<true, 256, 4, 1>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), G2::kSmemBytes, dev.device)) != FP8MM_OK) return st;
     kern<<<grid, kGemmThreads, G2::kSmemBytes, stream>>>(ta, tb, p);
@@ -227,15 +237,15 @@ static fp8mm_status launch_tiled(bool mx, const void* a, const void* b, const ui
 using P1 = PairCfg<false, 6, 2>;
 using P2 = PairCfg<true, 6, 1>;
 
-// Largest number of co-resident 2-CTA clusters of a pair kernel (cached).
-static fp8mm_status max_pairs(const void* kern, int smem, const DeviceInfo& dev, int* out) {
-  static std::set<std::pair<const void*, int>> done;
-  static int cached[2][64];
-  const int which = (kern == reinterpret_cast<const void*>(gemm_pair_kernel<true, 6, 1>)) ? 1 : 0;
+// Largest number of co-resident 2-CTA clusters of a pair kernel (cached per
+// kernel and device).
+static fp8mm_status max_pairs(const void* kern, int smem, int threads, const DeviceInfo& dev, int* out) {
+  static std::map<std::pair<const void*, int>, int> cached;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (done.count({kern, dev.device})) {
-      *out = cached[which][dev.device];
+    auto it = cached.find({kern, dev.device});
+    if (it != cached.end()) {
+      *out = it->second;
       return FP8MM_OK;
     }
   }
@@ -246,7 +256,7 @@ static fp8mm_status max_pairs(const void* kern, int smem, const DeviceInfo& dev,
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(2 * (dev.sms / 2), 1, 1);
-  cfg.blockDim = dim3(which ? P2::kThreads : P1::kThreads, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -255,15 +265,16 @@ static fp8mm_status max_pairs(const void* kern, int smem, const DeviceInfo& dev,
   if (e != cudaSuccess) return cuda_fail(e);
   if (n <= 0) n = 1;
   std::lock_guard<std::mutex> lock(g_mu);
-  cached[which][dev.device] = n;
-  done.insert({kern, dev.device});
+  cached[{kern, dev.device}] = n;
   *out = n;
   return FP8MM_OK;
 }
 
+// c8 != nullptr (mode 1 only): E4M3 output c8 = E4M3(C / *s_out) instead of bf16 c.
 static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uint8_t* sfa, const uint8_t* sfb,
                                 int64_t m, int64_t n, int64_t k, const float* sa, const float* sb, void* c,
-                                int64_t ldc, cudaStream_t stream, const DeviceInfo& dev) {
+                                int64_t ldc, cudaStream_t stream, const DeviceInfo& dev, uint8_t* c8 = nullptr,
+                                const float* s_out = nullptr) {
   CUtensorMap ta, tb, tsa, tsb;
   fp8mm_status st = make_map(&ta, a, k, m, 128);
   if (st != FP8MM_OK) return st;
@@ -292,12 +303,16 @@ static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uin
   p.n_kc = static_cast<int>(cdiv(k, 128));
   p.sfb_row_tiles = static_cast<int>(cdiv(n, 128));
   p.timeout_ns = wait_timeout_ns();
+  p.c8 = c8;
+  p.s_out = s_out;
   const void* kern = mx ? reinterpret_cast<const void*>(gemm_pair_kernel<true, 6, 1>)
-                        : reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2>);
+                     : c8 ? reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2, true>)
+                          : reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2>);
   const int smem = mx ? P2::kSmemBytes : P1::kSmemBytes;
+  const int threads = mx ? P2::kThreads : P1::kThreads;
   if ((st = ensure_smem(kern, smem, dev.device)) != FP8MM_OK) return st;
   int pairs = 0;
-  if ((st = max_pairs(kern, smem, dev, &pairs)) != FP8MM_OK) return st;
+  if ((st = max_pairs(kern, smem, threads, dev, &pairs)) != FP8MM_OK) return st;
   pairs = std::min(pairs, p.num_tiles);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -306,13 +321,14 @@ static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uin
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(mx ? P2::kThreads : P1::kThreads, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = mx ? cudaLaunchKernelEx(&cfg, gemm_pair_kernel<true, 6, 1>, ta, tb, tsa, tsb, p)
-                     : cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false, 6, 2>, ta, tb, tsa, tsb, p);
+  cudaError_t e = mx   ? cudaLaunchKernelEx(&cfg, gemm_pair_kernel<true, 6, 1>, ta, tb, tsa, tsb, p)
+                  : c8 ? cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false, 6, 2, true>, ta, tb, tsa, tsb, p)
+                       : cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false, 6, 2>, ta, tb, tsa, tsb, p);
   if (e != cudaSuccess) return cuda_fail(e);
   return launched();
 }
@@ -518,6 +534,47 @@ fp8mm_status fp8_quantize_rowwise(const void* x_bf16, int64_t rows, int64_t k, i
   return st != FP8MM_OK ? st : launched();
 }
 
+fp8mm_status fp8_tensor_scale(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, float* scale,
+                              void* stream) {
+  if (rows < 0 || k < 0 || k % 8 != 0 || (k > 0 && ld_x < k)) return FP8MM_ERR_SHAPE;
+  if (rows * (k / 8) > int64_t{0xFFFFFFFF}) return FP8MM_ERR_SHAPE;
+  if (scale == nullptr || (rows > 0 && k > 0 && x_bf16 == nullptr)) return FP8MM_ERR_NULL;
+  if (!aligned(scale, 4) || (rows > 0 && k > 0 && (!aligned(x_bf16, 16) || ld_x % 8 != 0))) return FP8MM_ERR_ALIGN;
+  DeviceInfo dev;
+  fp8mm_status st = current_device(&dev);
+  if (st != FP8MM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(scale, 0, sizeof(float), s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (rows > 0 && k > 0) {
+    const int64_t vecs = rows * (k / 8);
+    const int grid = static_cast<int>(std::min<int64_t>(cdiv(vecs, kTensorThreads), static_cast<int64_t>(dev.sms) * 8));
+    st = launch_pdl(tensor_amax_kernel, dim3(grid), dim3(kTensorThreads), 0, s,
+                    static_cast<const __nv_bfloat16*>(x_bf16), rows, k, ld_x, reinterpret_cast<unsigned*>(scale));
+    if (st != FP8MM_OK) return st;
+  }
+  st = launch_pdl(tensor_scale_finalize_kernel, dim3(1), dim3(1), 0, s, scale);
+  return st != FP8MM_OK ? st : launched();
+}
+
+fp8mm_status fp8_quantize_static(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, const float* scale,
+                                 void* q_e4m3, int64_t ld_q, void* stream) {
+  if (rows < 0 || k < 0 || k % 8 != 0) return FP8MM_ERR_SHAPE;
+  if (rows == 0 || k == 0) return FP8MM_OK;
+  if (ld_x < k || ld_q < k || rows * (k / 8) > int64_t{0xFFFFFFFF}) return FP8MM_ERR_SHAPE;
+  if (x_bf16 == nullptr || q_e4m3 == nullptr || scale == nullptr) return FP8MM_ERR_NULL;
+  if (!aligned(x_bf16, 16) || !aligned(q_e4m3, 8) || !aligned(scale, 4) || ld_x % 8 != 0 || ld_q % 8 != 0)
+    return FP8MM_ERR_ALIGN;
+  DeviceInfo dev;
+  fp8mm_status st = current_device(&dev);
+  if (st != FP8MM_OK) return st;
+  const int64_t vecs = rows * (k / 8);
+  const int grid = static_cast<int>(std::min<int64_t>(cdiv(vecs, kTensorThreads), static_cast<int64_t>(dev.sms) * 8));
+  st = launch_pdl(quant_static_kernel, dim3(grid), dim3(kTensorThreads), 0, static_cast<cudaStream_t>(stream),
+                  static_cast<const __nv_bfloat16*>(x_bf16), rows, k, ld_x, scale, static_cast<uint8_t*>(q_e4m3), ld_q);
+  return st != FP8MM_OK ? st : launched();
+}
+
 fp8mm_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, void* q_e4m3, int64_t ld_q,
                             uint8_t* sf, void* stream) {
   if (rows < 0 || k < 0 || k % 32 != 0 || ld_x < k || ld_q < k) return FP8MM_ERR_SHAPE;
@@ -540,12 +597,12 @@ fp8mm_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
 }
 
 static fp8mm_status check_gemm_common(const void* a, const void* b, int64_t m, int64_t n, int64_t k, const void* c,
-                                      int64_t ldc, int64_t k_granule) {
+                                      int64_t ldc, int64_t k_granule, uintptr_t c_align = 2) {
   if (m < 0 || n < 0 || k < 0 || k % k_granule != 0 || ldc < n) return FP8MM_ERR_SHAPE;
   if (m > INT32_MAX / 2 || n > INT32_MAX / 2 || k > INT32_MAX / 2) return FP8MM_ERR_SHAPE;
   if (m == 0 || n == 0) return FP8MM_OK;
   if (c == nullptr || (k > 0 && (a == nullptr || b == nullptr))) return FP8MM_ERR_NULL;
-  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(c, 2)) return FP8MM_ERR_ALIGN;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(c, c_align)) return FP8MM_ERR_ALIGN;
   return FP8MM_OK;
 }
 
@@ -572,6 +629,34 @@ fp8mm_status fp8_gemm(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t
   const bool pair = (kind == FP8MM_KERNEL_TILED_2SM) || (kind != FP8MM_KERNEL_TILED_1SM && m >= 256);
   if (pair) return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev);
   return launch_tiled(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev);
+}
+
+fp8mm_status fp8_gemm_e4m3_out(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t n, int64_t k,
+                               const float* scale_a, const float* scale_b, const float* scale_out, void* c_e4m3,
+                               int64_t ldc, const fp8mm_opts* opt, void* stream) {
+  fp8mm_status st = check_gemm_common(a_e4m3, b_e4m3, m, n, k, c_e4m3, ldc, 16, 1);
+  if (st != FP8MM_OK || m == 0 || n == 0) return st;
+  if (scale_out == nullptr || (k > 0 && (scale_a == nullptr || scale_b == nullptr))) return FP8MM_ERR_NULL;
+  if (!aligned(scale_a, 4) || !aligned(scale_b, 4) || !aligned(scale_out, 4)) return FP8MM_ERR_ALIGN;
+  if (opt != nullptr && (opt->kernel == FP8MM_KERNEL_SMALL_M || opt->kernel < FP8MM_KERNEL_AUTO ||
+                         opt->kernel > FP8MM_KERNEL_TILED_2SM))
+    return FP8MM_ERR_SHAPE;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != FP8MM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (k == 0) {  // C = 0 encodes to 0x00
+    cudaError_t e = cudaMemset2DAsync(c_e4m3, static_cast<size_t>(ldc), 0, static_cast<size_t>(n),
+                                      static_cast<size_t>(m), s);
+    return e == cudaSuccess ? FP8MM_OK : cuda_fail(e);
+  }
+  const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
+  auto* c8 = static_cast<uint8_t*>(c_e4m3);
+  const bool pair = (kind == FP8MM_KERNEL_TILED_2SM) || (kind != FP8MM_KERNEL_TILED_1SM && m >= 256);
+  if (pair)
+    return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, nullptr, ldc, s, dev, c8,
+                       scale_out);
+  return launch_tiled(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, nullptr, ldc, s, dev, c8,
+                      scale_out);
 }
 
 fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e4m3, const uint8_t* sf_b, int64_t m,
@@ -636,6 +721,50 @@ fp8mm_status mxfp8_quantize_gemm(const void* a_bf16, int64_t lda, const void* b_
   uint8_t* sfx = tail + align256(static_cast<size_t>(m * k));
   if ((st = mxfp8_quantize(a_bf16, m, k, lda, xq, k, sfx, stream)) != FP8MM_OK) return st;
   return launch_small_m(xq, sfx, b_e4m3, sf_b, m, n, k, c_bf16, ldc, opt, s, dev);
+}
+
+fp8mm_status concat_mla_k(const void* k_nope, const void* k_rope, void* k_out, int64_t num_tokens,
+                          int64_t num_heads, int64_t nope_dim, int64_t rope_dim, int64_t elem_bytes,
+                          int64_t nope_stride_t, int64_t nope_stride_h, int64_t rope_stride_t,
+                          int64_t rope_stride_h, int64_t out_stride_t, int64_t out_stride_h, void* stream) {
+  if (num_tokens < 0 || num_heads < 0 || nope_dim <= 0 || rope_dim <= 0) return FP8MM_ERR_SHAPE;
+  if (elem_bytes != 1 && elem_bytes != 2) return FP8MM_ERR_SHAPE;
+  if (num_tokens == 0 || num_heads == 0) return FP8MM_OK;
+  const int64_t nope_b = nope_dim * elem_bytes, rope_b = rope_dim * elem_bytes;
+  const int64_t row_chunks = (nope_b + rope_b) / 16;
+  if (nope_b % 16 != 0 || rope_b % 16 != 0) return FP8MM_ERR_ALIGN;
+  if (num_tokens * num_heads > (int64_t{1} << 31) || num_tokens * num_heads * row_chunks > int64_t{0xFFFFFFFF})
+    return FP8MM_ERR_SHAPE;
+  if (nope_stride_h < nope_dim || out_stride_h < nope_dim + rope_dim || rope_stride_h < 0 ||
+      (rope_stride_h > 0 && rope_stride_h < rope_dim) || nope_stride_t < 0 || rope_stride_t < 0 ||
+      out_stride_t < nope_dim + rope_dim)
+    return FP8MM_ERR_SHAPE;
+  if (k_nope == nullptr || k_rope == nullptr || k_out == nullptr) return FP8MM_ERR_NULL;
+  const int64_t strides[6] = {nope_stride_t, nope_stride_h, rope_stride_t, rope_stride_h, out_stride_t, out_stride_h};
+  for (int64_t st : strides)
+    if ((st * elem_bytes) % 16 != 0) return FP8MM_ERR_ALIGN;
+  if (!aligned(k_nope, 16) || !aligned(k_rope, 16) || !aligned(k_out, 16)) return FP8MM_ERR_ALIGN;
+  DeviceInfo dev;
+  fp8mm_status st = current_device(&dev);
+  if (st != FP8MM_OK) return st;
+  ConcatArgs p{};
+  p.nope = static_cast<const uint8_t*>(k_nope);
+  p.rope = static_cast<const uint8_t*>(k_rope);
+  p.out = static_cast<uint8_t*>(k_out);
+  p.heads = static_cast<uint32_t>(num_heads);
+  p.nope_chunks = static_cast<uint32_t>(nope_b / 16);
+  p.row_chunks = static_cast<uint32_t>(row_chunks);
+  p.total_chunks = static_cast<uint32_t>(num_tokens * num_heads * row_chunks);
+  p.nope_st = nope_stride_t * elem_bytes;
+  p.nope_sh = nope_stride_h * elem_bytes;
+  p.rope_st = rope_stride_t * elem_bytes;
+  p.rope_sh = rope_stride_h * elem_bytes;
+  p.out_st = out_stride_t * elem_bytes;
+  p.out_sh = out_stride_h * elem_bytes;
+  const int grid = static_cast<int>(
+      std::min<int64_t>(cdiv(static_cast<int64_t>(p.total_chunks), kConcatThreads), static_cast<int64_t>(dev.sms) * 8));
+  st = launch_pdl(concat_mla_k_kernel, dim3(grid), dim3(kConcatThreads), 0, static_cast<cudaStream_t>(stream), p);
+  return st != FP8MM_OK ? st : launched();
 }
 
 unsigned int fp8mm_last_device_error(void) {

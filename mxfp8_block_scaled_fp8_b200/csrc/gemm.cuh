@@ -17,13 +17,16 @@
 //               the scale chunks) per 128-byte K slab, commits to free the slab.
 //   warps 2..9  epilogue: each drains half a tile row-block of the fp32
 //               accumulator into registers (tcgen05.ld, one wait), frees the
-//               accumulator, then scales, converts to bf16 RNE and stores.
+//               accumulator, then scales, converts to bf16 RNE and stores
+//               (or, with kOut8 in mode 1, E4M3 codes of C / scale_out: the
+//               FP8 output of listing 1's C_fp8 for the next layer).
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace fp8mm {
 
@@ -39,6 +42,8 @@ struct GemmArgs {
   int tiles_m, tiles_n, num_tiles;
   __nv_bfloat16* c;
   int64_t ldc;
+  uint8_t* c8;               // kOut8: E4M3 output (row stride ldc bytes)
+  const float* s_out;        // kOut8: output scale (device scalar)
   const float* sa;           // mode 1
   const float* sb;
   const uint8_t* sfa;        // mode 2 (library scale layout)
@@ -47,6 +52,59 @@ struct GemmArgs {
   int sfb_row_tiles;         // ceil(n / 128): 128-row tiles present in sfb
   uint64_t timeout_ns;
 };
+
+// Epilogue store of one thread's 32 consecutive outputs v[0..31] of row `row`
+// from column col0: bf16 round-to-nearest-even into p.c, or with kOut8 the
+// E4M3 codes of v / s_out (quotient_sat, IEEE division when !fast) into p.c8.
+// Full 32-column runs whose address is 16-byte aligned use 16-byte stores;
+// ragged or unaligned runs store element by element.
+template <bool kOut8>
+__device__ __forceinline__ void store_out32(const GemmArgs& p, int row, int col0, const float (&v)[32], float s_out,
+                                            float r_out, bool fast) {
+  if (row >= p.m || col0 >= p.n) return;
+  if constexpr (kOut8) {
+    uint32_t w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float y[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) y[u] = fast ? quotient_sat(v[4 * j + u], s_out, r_out) : __fdiv_rn(v[4 * j + u], s_out);
+      w[j] = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(y[0], y[1]), __NV_SATFINITE, __NV_E4M3)) |
+             (static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(y[2], y[3]), __NV_SATFINITE, __NV_E4M3)) << 16);
+    }
+    uint8_t* dst = p.c8 + static_cast<int64_t>(row) * p.ldc + col0;
+    if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+      reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + j < p.n) dst[j] = static_cast<uint8_t>(w[j >> 2] >> (8 * (j & 3)));
+    }
+  } else {
+    uint32_t packed[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+      packed[j] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    __nv_bfloat16* dst = p.c + static_cast<int64_t>(row) * p.ldc + col0;
+    if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+        *reinterpret_cast<uint4*>(dst + q4 * 8) =
+            make_uint4(packed[4 * q4], packed[4 * q4 + 1], packed[4 * q4 + 2], packed[4 * q4 + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (col0 + j < p.n) {
+          const uint32_t w = packed[j >> 1];
+          *reinterpret_cast<uint16_t*>(dst + j) = static_cast<uint16_t>((j & 1) ? (w >> 16) : (w & 0xFFFFu));
+        }
+      }
+    }
+  }
+}
 
 template <bool kMX, int kBN, int kStages, int kAccStages>
 struct GemmCfg {
@@ -85,7 +143,7 @@ __device__ __forceinline__ void tile_coords(int t, const GemmArgs& p, int& mb, i
   nb = r / gm;
 }
 
-template <bool kMX, int kBN, int kStages, int kAccStages>
+template <bool kMX, int kBN, int kStages, int kAccStages, bool kOut8 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const GemmArgs p) {
@@ -238,6 +296,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int sp = warp & 3;
     const int col_half = (warp - 2) >> 2;
     constexpr int kHalf = kBN / 2;
+    float s_out = 1.f, r_out = 1.f;
+    bool out_fast = true;
+    if constexpr (kOut8) {
+      s_out = __ldg(p.s_out);
+      r_out = __frcp_rn(s_out);
+      out_fast = quotient_fast_ok(s_out);
+    }
     static_assert(kHalf == 128, "epilogue assumes 256-column tiles");
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -270,35 +335,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int col0 = nb * kBN + col_half * kHalf + ch * 32;
         float sbv = 1.f;
         if constexpr (!kMX) sbv = (col0 + lane < p.n) ? __ldg(p.sb + col0 + lane) : 0.f;
-        uint32_t packed[16];
+        float v[32];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float v0 = __uint_as_float(r[ch][2 * j]);
-          float v1 = __uint_as_float(r[ch][2 * j + 1]);
-          if constexpr (!kMX) {
-            v0 = v0 * s_row * __shfl_sync(0xFFFFFFFFu, sbv, 2 * j);
-            v1 = v1 * s_row * __shfl_sync(0xFFFFFFFFu, sbv, 2 * j + 1);
-          }
-          __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-          packed[j] = *reinterpret_cast<uint32_t*>(&h);
+        for (int j = 0; j < 32; ++j) {
+          v[j] = __uint_as_float(r[ch][j]);
+          if constexpr (!kMX) v[j] = v[j] * s_row * __shfl_sync(0xFFFFFFFFu, sbv, j);
         }
-        if (row < p.m && col0 < p.n) {
-          __nv_bfloat16* dst = p.c + static_cast<int64_t>(row) * p.ldc + col0;
-          if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-              *reinterpret_cast<uint4*>(dst + q4 * 8) =
-                  make_uint4(packed[4 * q4], packed[4 * q4 + 1], packed[4 * q4 + 2], packed[4 * q4 + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (col0 + j < p.n) {
-                const uint32_t w = packed[j >> 1];
-                *reinterpret_cast<uint16_t*>(dst + j) = static_cast<uint16_t>((j & 1) ? (w >> 16) : (w & 0xFFFFu));
-              }
-            }
-          }
-        }
+        store_out32<kOut8>(p, row, col0, v, s_out, r_out, out_fast);
       }
     }
   }

@@ -1,7 +1,7 @@
 // gemm2.cuh -- paired-SM tcgen05 GEMM (cta_group::2) for both scale modes.
 //
 // Same arithmetic as gemm.cuh (page "从 DeepGEMM 到 vLLM", listing 1 for the
-// per-token mode; page "[sglang] FlashInfer v0.6.7 MXFP8 Gemm 통합", section 2
+// per-token mode, with its bf16 or E4M3 output; page "[sglang] FlashInfer v0.6.7 MXFP8 Gemm 통합", section 2
 // for the block-scaled mode), computed by 2-CTA clusters on 256 x 256 output
 // tiles.  Each CTA of a pair loads its own 128-row half of the A tile and its
 // own 128-row half of the B tile; nothing is multicast.  Those loads complete
@@ -76,7 +76,7 @@ __device__ __forceinline__ void pair_tile_coords(int t, const GemmArgs& p, int& 
 // GemmArgs fields as in gemm.cuh, with tiles_m = ceil(m/256), tiles_n =
 // ceil(n/256).  tmSFA / tmSFB: 3-D maps over the scale layout viewed as
 // uint32 [n_rt][n_kc][128] (unused in per-token mode).
-template <bool kMX, int kStages, int kAccStages>
+template <bool kMX, int kStages, int kAccStages, bool kOut8 = false>
 __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
@@ -229,6 +229,13 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
     // ------------------------------------------------------ epilogue (both CTAs)
     const int sp = warp & 3;
     const int quarter = (warp - Cfg::kEpiWarp0) >> 2;  // 64-column slice of the 256-column tile
+    float s_out = 1.f, r_out = 1.f;
+    bool out_fast = true;
+    if constexpr (kOut8) {
+      s_out = __ldg(p.s_out);
+      r_out = __frcp_rn(s_out);
+      out_fast = quotient_fast_ok(s_out);
+    }
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = pair; t < p.num_tiles; t += npairs) {
@@ -260,35 +267,13 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
         const int col0 = nb * 256 + quarter * 64 + ch * 32;
         float sbv = 1.f;
         if constexpr (!kMX) sbv = (col0 + lane < p.n) ? __ldg(p.sb + col0 + lane) : 0.f;
-        uint32_t packed[16];
+        float v[32];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float v0 = __uint_as_float(r[ch][2 * j]);
-          float v1 = __uint_as_float(r[ch][2 * j + 1]);
-          if constexpr (!kMX) {
-            v0 = v0 * s_row * __shfl_sync(0xFFFFFFFFu, sbv, 2 * j);
-            v1 = v1 * s_row * __shfl_sync(0xFFFFFFFFu, sbv, 2 * j + 1);
-          }
-          __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-          packed[j] = *reinterpret_cast<uint32_t*>(&h);
+        for (int j = 0; j < 32; ++j) {
+          v[j] = __uint_as_float(r[ch][j]);
+          if constexpr (!kMX) v[j] = v[j] * s_row * __shfl_sync(0xFFFFFFFFu, sbv, j);
         }
-        if (row < p.m && col0 < p.n) {
-          __nv_bfloat16* dst = p.c + static_cast<int64_t>(row) * p.ldc + col0;
-          if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-              *reinterpret_cast<uint4*>(dst + q4 * 8) =
-                  make_uint4(packed[4 * q4], packed[4 * q4 + 1], packed[4 * q4 + 2], packed[4 * q4 + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (col0 + j < p.n) {
-                const uint32_t w = packed[j >> 1];
-                *reinterpret_cast<uint16_t*>(dst + j) = static_cast<uint16_t>((j & 1) ? (w >> 16) : (w & 0xFFFFu));
-              }
-            }
-          }
-        }
+        store_out32<kOut8>(p, row, col0, v, s_out, r_out, out_fast);
       }
     }
   }

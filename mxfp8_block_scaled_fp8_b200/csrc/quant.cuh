@@ -87,6 +87,17 @@ __device__ __forceinline__ bool quotient_fast_ok(float s) {
   return s >= 0x1p-80f && s <= 0x1p126f;
 }
 
+// x / s where x / s may lie far beyond the E4M3 range (a static scale, a GEMM
+// output): an approximation x * r above 1024 means the quotient is past 464
+// and saturates to 448 whatever its exact value, so +-1024 is returned (this
+// also covers x * r overflowing, where the correction would give NaN);
+// otherwise quotient_rn.  For bf16 x the result is the IEEE quotient or
+// saturates like it; for fp32 x (GEMM outputs) it is within one fp32 step.
+__device__ __forceinline__ float quotient_sat(float x, float s, float r) {
+  const float q0 = x * r;
+  return fabsf(q0) > 1024.f ? copysignf(1024.f, q0) : quotient_rn(x, s, r);
+}
+
 constexpr int kQ1Threads = 256;
 
 // One CTA per row (grid-stride over rows).  The row is held in registers
@@ -193,6 +204,68 @@ __global__ void __launch_bounds__(kQ1Threads) quant_rowwise_2pass_kernel(const _
       for (int j = 0; j < 8; ++j) f[j] = fast ? quotient_rn(f[j], s, r) : __fdiv_rn(f[j], s);
       *reinterpret_cast<uint2*>(qr + idx * 8) = f32x8_to_e4m3(f);
     }
+  }
+}
+
+// ------------------------------------------------------------------ per tensor
+
+// Per-tensor scale (page "FP8 推理基础设施（五）：从 DeepGEMM 到 vLLM", listing 3:
+// one scale per tensor, max|x| / 448), in two steps: every warp takes the
+// exact maximum of |x| over its vectors (an unsigned 16-bit max over the
+// sign-cleared bf16 bits) and folds it into *word with atomicMax (the word
+// was zeroed; bf16 bits << 16 are the fp32 bits of the maximum, whose integer
+// order is their value order); then one thread turns it into
+// s = amax / 448 (IEEE division), 1 for an all-zero tensor.
+constexpr int kTensorThreads = 256;
+
+__global__ void __launch_bounds__(kTensorThreads) tensor_amax_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                                                    int64_t k, int64_t ld_x, unsigned* word) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const uint32_t vpr = static_cast<uint32_t>(k / 8);  // 16-byte vectors per row
+  const uint32_t total = static_cast<uint32_t>(rows) * vpr;  // < 2^32 (checked by the host)
+  uint32_t m = 0;
+  for (uint32_t v = blockIdx.x * kTensorThreads + threadIdx.x; v < total; v += gridDim.x * kTensorThreads) {
+    const uint32_t r = v / vpr;
+    const uint4 w = ld_stream_16(x + static_cast<int64_t>(r) * ld_x + (v - r * vpr) * 8);
+    m = __vmaxu2(__vmaxu2(m, w.x & 0x7FFF7FFFu),
+                 __vmaxu2(w.y & 0x7FFF7FFFu, __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
+  }
+  m = max(m & 0xFFFFu, m >> 16) << 16;
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(word, m);
+}
+
+__global__ void tensor_scale_finalize_kernel(float* scale) {
+  griddep_wait();
+  const float amax = *scale;  // the maximum's bits, left by tensor_amax_kernel
+  *scale = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 448.f);
+}
+
+// Static-scale quantizer: q = E4M3_RNE_sat(fp32(x / s)) with one fp32 scale
+// for the whole tensor (a calibrated per-tensor scale; also the FP8 KV-cache
+// quantizer).  Grid-stride over 16-byte vectors; the quotient is quotient_sat
+// (the IEEE quotient, or saturated like it) when quotient_fast_ok(s), else
+// an IEEE division.
+__global__ void __launch_bounds__(kTensorThreads) quant_static_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                                                     int64_t k, int64_t ld_x,
+                                                                     const float* __restrict__ scale,
+                                                                     uint8_t* __restrict__ q, int64_t ld_q) {
+  griddep_launch_dependents();
+  griddep_wait();  // the scale and x may be written by the preceding kernel
+  const float s = *scale;
+  const float r = __frcp_rn(s);
+  const bool fast = quotient_fast_ok(s);
+  const uint32_t vpr = static_cast<uint32_t>(k / 8);
+  const uint32_t total = static_cast<uint32_t>(rows) * vpr;  // < 2^32 (checked by the host)
+  for (uint32_t v = blockIdx.x * kTensorThreads + threadIdx.x; v < total; v += gridDim.x * kTensorThreads) {
+    const uint32_t row = v / vpr;
+    const uint32_t c8 = v - row * vpr;
+    float f[8];
+    bf16x8_to_f32(ld_stream_16(x + static_cast<int64_t>(row) * ld_x + c8 * 8), f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = fast ? quotient_sat(f[j], s, r) : __fdiv_rn(f[j], s);
+    *reinterpret_cast<uint2*>(q + static_cast<int64_t>(row) * ld_q + c8 * 8) = f32x8_to_e4m3(f);
   }
 }
 

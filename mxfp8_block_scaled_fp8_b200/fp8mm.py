@@ -50,8 +50,12 @@ _SIGNATURES = {
     "fp8_quantize_rowwise": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P], ctypes.c_int),
     "mxfp8_quantize": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P], ctypes.c_int),
     "fp8_gemm": ([_P, _P, _I64, _I64, _I64, _P, _P, _P, _I64, ctypes.POINTER(Opts), _P], ctypes.c_int),
+    "fp8_tensor_scale": ([_P, _I64, _I64, _I64, _P, _P], ctypes.c_int),
+    "fp8_quantize_static": ([_P, _I64, _I64, _I64, _P, _P, _I64, _P], ctypes.c_int),
+    "fp8_gemm_e4m3_out": ([_P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I64, ctypes.POINTER(Opts), _P], ctypes.c_int),
     "mxfp8_gemm": ([_P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, ctypes.POINTER(Opts), _P], ctypes.c_int),
     "mxfp8_quantize_gemm": ([_P, _I64, _P, _P, _I64, _I64, _I64, _P, _I64, ctypes.POINTER(Opts), _P], ctypes.c_int),
+    "concat_mla_k": ([_P, _P, _P] + [_I64] * 11 + [_P], ctypes.c_int),
     "fp8mm_sf_bytes": ([_I64, _I64], ctypes.c_size_t),
     "fp8mm_sf_offset": ([_I64, _I64, _I64, _I64], ctypes.c_int64),
     "fp8mm_sf_to_canonical": ([_P, _I64, _I64, _P], ctypes.c_int),
@@ -138,6 +142,54 @@ def fp8_gemm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: t
     opts = Opts(None, 0, kernel, 0, 0)
     _check("fp8_gemm", lib().fp8_gemm(a.data_ptr(), b.data_ptr(), m, n, k, scale_a.data_ptr(), scale_b.data_ptr(),
                                       c.data_ptr(), _ld(c, "c"), ctypes.byref(opts), _stream(stream)))
+    return c
+
+
+# ----------------------------------------------------------------- per tensor, FP8 out
+
+def fp8_tensor_scale(x: torch.Tensor, scale: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """bf16 [rows, k] -> fp32 [1] device scale = max|x| / 448 over the whole tensor (1 if all zero)."""
+    _need(x, torch.bfloat16, "x")
+    rows, k = x.shape
+    if scale is None:
+        scale = torch.empty((1,), dtype=torch.float32, device=x.device)
+    _check("fp8_tensor_scale", lib().fp8_tensor_scale(x.data_ptr(), rows, k, _ld(x, "x") if k else k,
+                                                      scale.data_ptr(), _stream(stream)))
+    return scale
+
+
+def fp8_quantize_static(x: torch.Tensor, scale: torch.Tensor, q: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """bf16 [rows, k] and a device fp32 scale -> E4M3 codes uint8 [rows, k] of x / scale."""
+    _need(x, torch.bfloat16, "x"); _need(scale, torch.float32, "scale")
+    rows, k = x.shape
+    if q is None:
+        q = torch.empty((rows, k), dtype=torch.uint8, device=x.device)
+    q = _u8(q)
+    _check("fp8_quantize_static", lib().fp8_quantize_static(x.data_ptr(), rows, k, _ld(x, "x"), scale.data_ptr(),
+                                                            q.data_ptr(), _ld(q, "q"), _stream(stream)))
+    return q
+
+
+def fp8_gemm_e4m3_out(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
+                      scale_out: torch.Tensor, c: torch.Tensor | None = None, kernel: int = KERNEL_AUTO,
+                      stream=None) -> torch.Tensor:
+    """E4M3 codes uint8 [m, n] of diag(scale_a) (A x B^T) diag(scale_b) / scale_out."""
+    a, b = _u8(a), _u8(b)
+    _need(a, torch.uint8, "a"); _need(b, torch.uint8, "b")
+    _need(scale_a, torch.float32, "scale_a"); _need(scale_b, torch.float32, "scale_b")
+    _need(scale_out, torch.float32, "scale_out")
+    m, k = a.shape
+    n = b.shape[0]
+    if b.shape[1] != k or not (a.is_contiguous() and b.is_contiguous()):
+        raise ValueError("a [m,k] and b [n,k] must be contiguous with the same k")
+    if c is None:
+        c = torch.empty((m, n), dtype=torch.uint8, device=a.device)
+    c = _u8(c)
+    opts = Opts(None, 0, kernel, 0, 0)
+    _check("fp8_gemm_e4m3_out", lib().fp8_gemm_e4m3_out(
+        a.data_ptr(), b.data_ptr(), m, n, k, scale_a.data_ptr(), scale_b.data_ptr(), scale_out.data_ptr(),
+        c.data_ptr(), _ld(c, "c"), ctypes.byref(opts), _stream(stream)))
     return c
 
 
@@ -233,6 +285,32 @@ def mxfp8_quantize_gemm(a: torch.Tensor, b: torch.Tensor, sf_b: torch.Tensor, c:
         a.data_ptr(), _ld(a, "a"), b.data_ptr(), sf_b.data_ptr(), m, n, k, c.data_ptr(), _ld(c, "c"),
         ctypes.byref(opts), _stream(stream)))
     return c
+
+
+# ----------------------------------------------------------------- KV cache
+
+def concat_mla_k(k_nope: torch.Tensor, k_rope: torch.Tensor, out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """k_nope [T, H, nope], k_rope [T, H or 1, rope] (1 = one rope vector per token for all heads)
+    -> out [T, H, nope + rope]; 1-byte (float8 / uint8) or 2-byte elements, any 16-byte-aligned strides."""
+    if k_nope.dim() != 3 or k_rope.dim() != 3 or not k_nope.is_cuda or not k_rope.is_cuda:
+        raise ValueError("k_nope and k_rope must be 3-D CUDA tensors")
+    if k_nope.element_size() != k_rope.element_size() or k_nope.dtype != k_rope.dtype:
+        raise TypeError("k_nope and k_rope must have the same dtype")
+    T, H, dn = k_nope.shape
+    dr = k_rope.shape[2]
+    if k_rope.shape[0] != T or k_rope.shape[1] not in (1, H) or k_nope.stride(2) != 1 or k_rope.stride(2) != 1:
+        raise ValueError("k_rope must be [T, H or 1, rope] with unit element stride, k_nope unit element stride")
+    if out is None:
+        out = torch.empty((T, H, dn + dr), dtype=k_nope.dtype, device=k_nope.device)
+    if out.shape != (T, H, dn + dr) or out.stride(2) != 1 or out.dtype != k_nope.dtype:
+        raise ValueError("out must be [T, H, nope + rope] of the input dtype with unit element stride")
+    rope_sh = 0 if k_rope.shape[1] == 1 else k_rope.stride(1)
+    _check("concat_mla_k", lib().concat_mla_k(
+        k_nope.data_ptr(), k_rope.data_ptr(), out.data_ptr(), T, H, dn, dr, k_nope.element_size(),
+        k_nope.stride(0), k_nope.stride(1), k_rope.stride(0), rope_sh, out.stride(0), out.stride(1),
+        _stream(stream)))
+    return out
 
 
 # ----------------------------------------------------------------- misc

@@ -71,6 +71,21 @@ def test_argument_errors_without_a_gpu():
     assert Q(P(fake), 64, P(fake), P(fake), 4, 4, 64, P(fake), 8, ctypes.byref(tiled), None) == 2
     assert Q(None, 64, None, None, 0, 4, 64, None, 8, None, None) == 0                 # m == 0
     assert Q(P(fake), 64, P(fake), P(fake), 9, 4, 64, P(fake), 8, None, None) == 6      # m > 8 needs a workspace
+    # per-tensor scale, static quantizer, E4M3-output GEMM, MLA key concatenation
+    assert L.fp8_tensor_scale(P(fake), 4, 12, 16, P(fake), None) == 2                       # k % 8
+    assert L.fp8_tensor_scale(P(fake), 4, 16, 16, None, None) == 1                          # scale
+    assert L.fp8_quantize_static(P(fake), 4, 16, 16, None, P(fake), 16, None) == 1          # scale
+    assert L.fp8_quantize_static(P(fake), 4, 16, 16, P(fake), P(fake + 4), 16, None) == 3   # q alignment
+    assert L.fp8_quantize_static(None, 0, 16, 16, None, None, 16, None) == 0                # empty
+    E = L.fp8_gemm_e4m3_out
+    assert E(P(fake), P(fake), 4, 4, 15, P(fake), P(fake), P(fake), P(fake), 8, None, None) == 2      # k % 16
+    assert E(P(fake), P(fake), 4, 4, 16, P(fake), P(fake), None, P(fake), 8, None, None) == 1         # scale_out
+    assert E(P(fake), P(fake), 4, 4, 16, P(fake), P(fake), P(fake), P(fake + 1), 8, None, None) != 3  # any c alignment
+    C = L.concat_mla_k
+    assert C(P(fake), P(fake), P(fake), 2, 2, 128, 64, 3, 256, 128, 64, 0, 384, 192, None) == 2       # elem bytes
+    assert C(P(fake), P(fake), P(fake), 2, 2, 120, 64, 1, 240, 120, 64, 0, 368, 184, None) == 3       # 120-byte rows
+    assert C(P(fake + 8), P(fake), P(fake), 2, 2, 128, 64, 1, 256, 128, 64, 0, 384, 192, None) == 3   # base
+    assert C(None, None, None, 0, 2, 128, 64, 1, 256, 128, 64, 0, 384, 192, None) == 0                # no tokens
     # empty problems are no-ops and need no device
     assert L.fp8_gemm(None, None, 0, 4, 16, None, None, None, 8, None, None) == 0
     assert L.mxfp8_quantize(None, 0, 64, 64, None, 64, None, None) == 0

@@ -14,6 +14,7 @@ import oracle
 from tests import test_oracle_formats as F
 from tests import test_oracle_gemm as G
 from tests import test_oracle_quant as Q
+from tests import test_oracle_static_concat as S
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 
@@ -21,7 +22,12 @@ MUTANTS = {
     "ties_away_from_even": ("pick = (c % 2 == 0) ? c : c + 1;", "pick = c + 1;"),
     "mx_bias_off_by_one": ("ceil(log2(amax / 448.0)) + 127.0", "ceil(log2(amax / 448.0)) + 126.0"),
     "mx_floor_not_ceil": ("ceil(log2(amax / 448.0))", "floor(log2(amax / 448.0))"),
-    "rowwise_wrong_divisor": ("(double)amax / 448.0", "(double)amax / 480.0"),
+    "rowwise_wrong_divisor": ("float s = (amax == 0.0f) ? 1.0f : (float)((double)amax / 448.0);",
+                              "float s = (amax == 0.0f) ? 1.0f : (float)((double)amax / 480.0);"),
+    "tensor_scale_wrong_divisor": ("return (amax == 0.0f) ? 1.0f : (float)((double)amax / 448.0);",
+                                   "return (amax == 0.0f) ? 1.0f : (float)((double)amax / 480.0);"),
+    "static_scale_multiplied": ("bf16_to_float(c->x[r * c->ld_x + j]) / c->s;",
+                                "bf16_to_float(c->x[r * c->ld_x + j]) * c->s;"),
     "sign_dropped": ("signbit(v) ? 0x80 : 0x00", "0x00"),
     "overflow_to_nan": ("if (a >= 448.0) return sign | 0x7E;", "if (a >= 448.0) return sign | 0x7F;"),
     "b_scale_dropped": ("(double)g->sa[i] * (double)g->sb[j]", "(double)g->sa[i]"),
@@ -39,6 +45,10 @@ PINS = [
     G.test_all_ones_closed_form, G.test_selection_matrix_reproduces_rows_of_b,
     lambda o: G.test_mx_exact_against_integer_brute_force(o, 3, 4, 64),
     lambda o: G.test_rowwise_exact_against_integer_brute_force(o, 3, 5, 16),
+    lambda o: S.test_tensor_scale_is_the_largest_row_scale(),
+    lambda o: S.test_tensor_scale_closed_forms(3),
+    lambda o: S.test_static_with_power_of_two_scale_is_exact_scaling(-1),
+    lambda o: S.test_static_with_the_row_scale_is_the_row_quantizer(),
 ]
 
 
@@ -62,7 +72,7 @@ def test_pins_catch_planted_mistake(tmp_path, monkeypatch, orc, name):
     real = oracle.lib()
     mut = ctypes.CDLL(path)
     for fn in ("orc_e4m3_decode", "orc_e4m3_encode", "orc_mx_exponent", "orc_quantize_rowwise",
-               "orc_mx_quantize", "orc_gemm_rowwise", "orc_gemm_mx"):
+               "orc_mx_quantize", "orc_gemm_rowwise", "orc_gemm_mx", "orc_tensor_scale", "orc_quantize_static"):
         getattr(mut, fn).argtypes = getattr(real, fn).argtypes
         getattr(mut, fn).restype = getattr(real, fn).restype
     monkeypatch.setattr(oracle, "_lib", mut)
