@@ -400,26 +400,53 @@ def run_ours(args):
     ms_per_step = total_ms / args.steps
     value = job_tflops(FLOPS_PER_STEP, args.steps, ws, total_ms)
 
-    # end to end through the public API with host buffers: H2D of X, the two
-    # calls, D2H of C, all inside the timed region
+    # end to end through the public API with host buffers, pipelined the way a
+    # serving loop runs it: every step copies its X in from pinned host memory,
+    # runs mxfp8_quantize + mxfp8_gemm, and copies its full C back to pinned
+    # host memory, all inside the timed region.  The copies and the kernels
+    # are on three streams with two device buffer sets, so step i+1's upload
+    # and step i-1's readback overlap step i's kernels (PCIe is full duplex).
+    e2e_steps = max(4, min(args.steps, 10))
     x_host = x_cpu.pin_memory()
-    c_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    e2e_steps = max(2, min(args.steps, 5))
-    for _ in range(2):
-        x.copy_(x_host, non_blocking=True)
-        step()
-        c_host.copy_(c, non_blocking=True)
+    c_hosts = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_devs = [x, torch.empty_like(x)]
+    c_devs = [c, torch.empty_like(c)]
+    s_h2d, s_cmp, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def e2e_run(n):
+        h2d_ev = [torch.cuda.Event() for _ in range(n)]
+        cmp_ev = [torch.cuda.Event() for _ in range(n)]
+        d2h_ev = [torch.cuda.Event() for _ in range(n)]
+        for i in range(n):
+            b = i % 2
+            if i >= 2:
+                s_h2d.wait_event(cmp_ev[i - 2])            # x_devs[b] no longer read
+            with torch.cuda.stream(s_h2d):
+                x_devs[b].copy_(x_host, non_blocking=True)
+                h2d_ev[i].record(s_h2d)
+            s_cmp.wait_event(h2d_ev[i])
+            if i >= 2:
+                s_cmp.wait_event(d2h_ev[i - 2])            # c_devs[b] read back
+            with torch.cuda.stream(s_cmp):
+                fp8mm.mxfp8_quantize(x_devs[b], qx, sfx)
+                fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c_devs[b])
+                cmp_ev[i].record(s_cmp)
+            s_d2h.wait_event(cmp_ev[i])
+            with torch.cuda.stream(s_d2h):
+                c_hosts[b].copy_(c_devs[b], non_blocking=True)
+                d2h_ev[i].record(s_d2h)
+
+    torch.cuda.synchronize()
+    e2e_run(2)                                          # warm-up
     torch.cuda.synchronize()
     a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a_ev.record(stream)
-    for _ in range(e2e_steps):
-        x.copy_(x_host, non_blocking=True)
-        step()
-        c_host.copy_(c, non_blocking=True)
-    b_ev.record(stream)
+    a_ev.record(s_h2d)
+    e2e_run(e2e_steps)
+    b_ev.record(s_d2h)                                  # after every readback (each waited for its step)
     torch.cuda.synchronize()
     e2e_ms = a_ev.elapsed_time(b_ev) / e2e_steps
     e2e_ms = max_over_ranks(e2e_ms, dev)
+    del x_devs, c_devs
 
     rows = None
     if rank == 0 and not args.no_rows:
@@ -436,8 +463,9 @@ def run_ours(args):
                    "M": M, "N": N, "K": K, "parallelism": f"dp{ws} (independent replicas)",
                    "l2": "inputs larger than L2: X 128 MiB bf16 and Wq 172 MiB are re-read every step"},
         "e2e": {"value": job_tflops(FLOPS_PER_STEP, 1, ws, e2e_ms), "unit": "TFLOPS",
-                "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": c_host.numel() * 2,
-                "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": c_hosts[0].numel() * 2,
+                "ms_per_step": e2e_ms, "steps": e2e_steps,
+                "pipelining": "H2D, kernels and D2H on three streams with two device buffer sets"},
         "gpu_launches": 2 * args.steps,
         "kernels": {"mxfp8_quantize_ms": q_ms, "mxfp8_gemm_ms": g_ms},
         "roofline": {"bound": "tensor", "kernel": "gemm_pair_kernel<mx> (mxfp8_gemm, 256x256 tiles on 2-CTA clusters)", "achieved": achieved,
