@@ -330,17 +330,21 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
 #pragma unroll
       for (int j = 0; j < kNM; ++j)
         if (j < p.m) mine[j * 128 + nl] = __uint_as_float(r[j]);
-      __threadfence();
+      // The four warps' partial stores are ordered before one thread's
+      // acquire-release ticket increment at GPU scope (the barrier between
+      // them is CTA-scope release/acquire and release is cumulative); the
+      // last contributor's increment acquires every earlier contributor's
+      // stores, and the barrier after it hands them to its other threads.
       if (!epi_meet()) break;
       const int b_first = dec_owner(static_cast<int64_t>(t) * p.num_k, p);
       const int b_last = dec_owner(static_cast<int64_t>(t + 1) * p.num_k - 1, p);
       if (threadIdx.x == 64) {
-        const unsigned prev = atomicAdd(&p.tickets[t], 1u);
+        unsigned prev;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(&p.tickets[t]) : "memory");
         *last_flag = (prev == static_cast<unsigned>(b_last - b_first)) ? 1 : 0;
       }
       if (!epi_meet()) break;
       if (*last_flag) {
-        __threadfence();
         // Sum the contributors' partials in CTA order (fixed, so the result
         // does not depend on arrival order); kU contributors' loads are in
         // flight at a time.
