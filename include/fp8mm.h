@@ -14,6 +14,12 @@
  *           (section 1: one uint8 scale per 32 elements of K, [n, k // 32];
  *           section 2: the GEMM call on the quantized activation and the
  *           pre-processed weight).
+ * Around them: a per-tensor calibration scale, a static-scale quantizer and
+ * an fp8_gemm with E4M3 output (listing 3 as printed; listing 1's C_fp8); a
+ * decode GEMM from a bf16 activation that quantizes it in the kernel
+ * (mxfp8_quantize_gemm); and the FP8 key assembly of multi-head latent
+ * attention (concat_mla_k, page "[flashinfer] FlashInfer, FP8 지원으로 장문
+ * 컨텍스트 추론 성능을 극적으로 향상시키다").
  *
  * Conventions shared by every entry point
  *   - Pointers named *_bf16, *_e4m3, c, scale*, sf* are DEVICE pointers owned
