@@ -471,6 +471,7 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "kernel": "gemm_pair_kernel<mx> (mxfp8_gemm, 256x256 tiles on 2-CTA clusters)", "achieved": achieved,
                      "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
                      "traffic": _ncu_traffic("mxfp8_gemm_ffn_up"),
+                     "frac_of_sustained": achieved / (2.0 * peaks["bf16_tflops_sustained"]),
                      "peak_note": f"FP8 dense = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s "
                                   f"(nominal FP8/BF16 ratio); sustained-based peak "
                                   f"{2.0 * peaks['bf16_tflops_sustained']:.0f}",
