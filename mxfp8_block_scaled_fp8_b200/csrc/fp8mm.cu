@@ -385,12 +385,21 @@ static fp8mm_status launch_small_m_t(const CUtensorMap& tw, const CUtensorMap& t
   return launched();
 }
 
-// CTAs of the small-M kernel: the requested number, else one per SM but no
-// fewer than 4 K slabs per CTA (more CTAs would only add partial tiles to
-// reduce); never more than there are slabs, never fewer than the tiles.
+// CTAs of the small-M kernel: the requested number; else one per SM, or two
+// per SM when two fit (token tiles up to 32), the weight tiles are short
+// (<= 48 K slabs, so the finer split adds at most about one contributor per
+// tile) and every CTA keeps >= 8 slabs -- measured on B200, that makes the
+// 14336 x 4096 projection ~10 % faster while the 4096 x 14336 (112-slab
+// tiles) and 6144 x 4096 (~5 slabs per CTA) ones get slower; in every case no
+// fewer than 4 slabs per CTA, never more CTAs than slabs, never fewer than
+// the tiles.
 constexpr int64_t kMinSlabsPerCta = 4;
-static int small_m_ctas(int64_t units, int64_t n_tiles, int64_t requested, int64_t sms) {
-  int64_t g = requested > 0 ? requested : std::min<int64_t>(sms, std::max<int64_t>(n_tiles, cdiv(units, kMinSlabsPerCta)));
+static int small_m_ctas(int64_t units, int64_t n_tiles, int64_t num_k, int nm, int64_t requested, int64_t sms) {
+  int64_t g = requested;
+  if (g <= 0) {
+    const bool two_per_sm = nm <= 32 && num_k <= 48 && units >= 2 * sms * 8;
+    g = std::min<int64_t>(two_per_sm ? 2 * sms : sms, std::max<int64_t>(n_tiles, cdiv(units, kMinSlabsPerCta)));
+  }
   g = std::min<int64_t>(g, units);
   return static_cast<int>(std::max<int64_t>(g, 1));
 }
@@ -418,7 +427,7 @@ static fp8mm_status launch_small_m(const void* a, const uint8_t* sfa, const void
   if (opt == nullptr || opt->workspace == nullptr) {
     p.ctas = p.n_tiles;  // one CTA per weight tile, whole K: no partial sums
   } else {
-    p.ctas = small_m_ctas(p.units, p.n_tiles, opt->small_m_ctas, dev.sms);
+    p.ctas = small_m_ctas(p.units, p.n_tiles, p.num_k, nm, opt->small_m_ctas, dev.sms);
     const size_t need = fp8mm_workspace_bytes(m, n, k, p.ctas);
     if (opt->workspace_bytes < need || !aligned(opt->workspace, 256)) return FP8MM_ERR_WORKSPACE;
     p.partials = static_cast<float*>(opt->workspace);
@@ -512,7 +521,7 @@ size_t fp8mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas) {
     cudaGetLastError();  // a host without a GPU leaves an error behind
   }
   const int64_t units = cdiv(n, 128) * cdiv(k, 128);
-  g = small_m_ctas(units, cdiv(n, 128), ctas, g);
+  g = small_m_ctas(units, cdiv(n, 128), cdiv(k, 128), small_m_tile(m), ctas, g);
   const size_t tickets = static_cast<size_t>(cdiv(n, 128)) * sizeof(unsigned);
   return small_m_partials_bytes(g, small_m_tile(m)) + ((tickets + 255) & ~size_t(255));
 }
