@@ -55,6 +55,7 @@ struct DecodeArgs {
   unsigned* tickets;   // [n_tiles], zero between calls
   uint64_t timeout_ns;
   int prefetch_w;      // weights may be read before the preceding kernel ends
+  int l2_ahead;        // slabs past the staged ones whose weights are prefetched into L2 at the start
   const __nv_bfloat16* x;  // kQX: bf16 activation [m, k]
   int64_t ldx;             // kQX: its row stride in elements
 };
@@ -184,6 +185,18 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
         mbar_arrive_expect_tx(&full[i], kTx);
         tma_load_2d(smem + Cfg::kOffW + i * Cfg::kWBytes, &tmW, &full[i], kb * 128, t * 128);
         bulk_load(smem + Cfg::kOffSfw + i * 512, p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u, &full[i]);
+        if (++kb == p.num_k) {
+          kb = 0;
+          ++t;
+        }
+      }
+      // The weights of the next l2_ahead slabs go to L2 now, so that HBM keeps
+      // streaming while the stages wait for the activation (and, under
+      // programmatic launch, for the preceding kernel).
+      const int64_t l2_end = npre + p.l2_ahead < nslabs ? npre + p.l2_ahead : nslabs;
+      for (int64_t i = npre; i < l2_end; ++i) {
+        tma_prefetch_l2_2d(&tmW, kb * 128, t * 128);
+        bulk_prefetch_l2(p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u);
         if (++kb == p.num_k) {
           kb = 0;
           ++t;

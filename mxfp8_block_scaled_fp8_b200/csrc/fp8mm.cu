@@ -385,6 +385,19 @@ static fp8mm_status launch_small_m_t(const CUtensorMap& tw, const CUtensorMap& t
   return launched();
 }
 
+// Slabs per CTA (past the staged ones) whose weights the small-M kernel
+// prefetches into L2 when it starts.  Only where two CTAs share an SM: the
+// next call's CTAs then start as this call's finish, and the prefetch keeps
+// HBM busy through this call's tail.  Measured on B200 (14336 x 4096, m <= 32,
+// back-to-back calls): 2 slabs ahead makes a call 2-5 % faster, 4 and more
+// slower.  With one CTA per SM the next call's CTAs sit beside this call's
+// from its start, and any prefetch only takes bandwidth from it.
+constexpr int64_t kL2AheadSlabs = 2;
+static int small_m_l2_ahead(int64_t units, int64_t ctas, int64_t sms) {
+  if (ctas <= sms) return 0;
+  return static_cast<int>(std::min<int64_t>(kL2AheadSlabs, cdiv(units, ctas)));
+}
+
 // CTAs of the small-M kernel: the requested number; else one per SM, or two
 // per SM when two fit (token tiles up to 32), the weight tiles are short
 // (<= 48 K slabs, so the finer split adds at most about one contributor per
@@ -434,6 +447,7 @@ static fp8mm_status launch_small_m(const void* a, const uint8_t* sfa, const void
     p.tickets = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(opt->workspace) +
                                             small_m_partials_bytes(p.ctas, nm));
   }
+  p.l2_ahead = small_m_l2_ahead(p.units, p.ctas, dev.sms);
   CUtensorMap tw, tx;
   fp8mm_status st = make_map(&tw, b, k, n, 128);
   if (st != FP8MM_OK) return st;
@@ -893,6 +907,7 @@ extern "C" fp8mm_status mxfp8_gemm_small_m_noalloc(const void* a_e4m3, const uin
   p.ctas = static_cast<int>(g);
   p.partials = reinterpret_cast<float*>(scratch);
   p.tickets = reinterpret_cast<unsigned*>(scratch + kNoAllocPartialBytes);
+  p.l2_ahead = small_m_l2_ahead(p.units, p.ctas, dev.sms);
   // the counters must start at zero; a previous call that stopped early may have left some set
   cudaError_t e = cudaMemsetAsync(p.tickets, 0, static_cast<size_t>(n_tiles) * sizeof(unsigned), s);
   if (e != cudaSuccess) return cuda_fail(e);
