@@ -51,6 +51,7 @@ struct GemmArgs {
   int n_kc;                  // scale chunks per 128-row tile = ceil(k / 128)
   int sfb_row_tiles;         // ceil(n / 128): 128-row tiles present in sfb
   uint64_t timeout_ns;
+  int group_m;               // paired-SM kernel: 256-row tiles per raster group
 };
 
 // Epilogue store of one thread's 32 consecutive outputs v[0..31] of row `row`

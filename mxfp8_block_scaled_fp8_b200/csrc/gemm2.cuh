@@ -38,7 +38,7 @@
 
 namespace fp8mm {
 
-constexpr int kPairGroupM = 8;     // 256-row tiles per raster group
+constexpr int kPairGroupM = 8;     // 256-row tiles per raster group (doubled for B larger than 64 MiB)
 
 template <bool kMX, int kStages, int kAccStages>
 struct PairCfg {
@@ -69,10 +69,10 @@ struct PairCfg {
 };
 
 __device__ __forceinline__ void pair_tile_coords(int t, const GemmArgs& p, int& mb, int& nb) {
-  const int per_group = kPairGroupM * p.tiles_n;
+  const int per_group = p.group_m * p.tiles_n;
   const int g = t / per_group;
-  const int first_m = g * kPairGroupM;
-  const int gm = min(p.tiles_m - first_m, kPairGroupM);
+  const int first_m = g * p.group_m;
+  const int gm = min(p.tiles_m - first_m, p.group_m);
   const int r = t - g * per_group;
   mb = first_m + r % gm;
   nb = r / gm;

@@ -93,6 +93,17 @@ def test_ffn_up_mx_sampled():
     run_mx(x, w, sample=_rows_cols(8192, 22016, 96, 96, 3), label="ffn_up 8192x22016x8192")
 
 
+def test_mx_tall_raster_groups_ragged():
+    """B above 64 MiB: the paired kernel rasters 16 rows of 256-row tiles
+    per group; 17 rows of tiles leave a last group of one (rows 4096..4199)."""
+    m, n, k = 4200, 8300, 8192
+    a = synthetic.random_bf16((m, k), seed=51)
+    bt = synthetic.random_bf16((n, k), seed=52, sigma=0.05)
+    rows, cols = _rows_cols(m, n, 40, 40, 5)
+    rows = np.unique(np.concatenate([rows, [4095, 4096, 4150]]))
+    run_mx(a, bt, sample=(rows, cols), label=f"mx {m}x{n}x{k}")
+
+
 # ------------------------------------------------------------ shapes and edges
 
 KERNELS = pytest.mark.parametrize("kernel", [fp8mm.KERNEL_TILED_1SM, fp8mm.KERNEL_TILED_2SM], ids=["1sm", "2sm"])
