@@ -411,17 +411,31 @@ static int small_m_l2_ahead(int64_t units, int64_t ctas, int64_t sms) {
 // CTAs of the small-M kernel: the requested number; else one per SM, or two
 // per SM when two fit (token tiles up to 32), the weight tiles are short
 // (<= 48 K slabs, so the finer split adds at most about one contributor per
-// tile) and every CTA keeps >= 8 slabs -- measured on B200, that makes the
-// 14336 x 4096 projection ~10 % faster while the 4096 x 14336 (112-slab
-// tiles) and 6144 x 4096 (~5 slabs per CTA) ones get slower; in every case no
-// fewer than 4 slabs per CTA, never more CTAs than slabs, never fewer than
-// the tiles.
+// tile) and every CTA keeps >= 8 slabs; in every case no fewer than 4 slabs
+// per CTA, never more CTAs than slabs, never fewer than the tiles.
+//
+// That count is replaced by a tile-aligned one -- s CTAs per weight tile,
+// with s dividing the tile's K slabs, so every CTA runs one segment inside
+// one tile and all contributors of a tile are equal -- when the largest such
+// count that fits the SMs (two per SM for token tiles up to 32) comes within
+// 80 % of it (16-token tiles) or 70 % (larger tiles, whose split-tile partials
+// cost more).  Measured on B200 with back-to-back calls (GEMM alone): 6144 x
+// 4096 at m <= 32 with 192 CTAs instead of 148 is 12-17 % faster, 4096 x
+// 14336 at m <= 8 with 256 instead of 148 8 %, at m = 64 with 128 instead of
+// 148 6 %, 14336 x 4096 at m = 32 with 224 instead of 296 5 % and at m = 64
+// with 112 instead of 148 9 %; at m <= 8 there 224 is 3 % slower than 296
+// (more bytes in flight outweigh the alignment for 16-token tiles).
 constexpr int64_t kMinSlabsPerCta = 4;
 static int small_m_ctas(int64_t units, int64_t n_tiles, int64_t num_k, int nm, int64_t requested, int64_t sms) {
   int64_t g = requested;
   if (g <= 0) {
     const bool two_per_sm = nm <= 32 && num_k <= 48 && units >= 2 * sms * 8;
     g = std::min<int64_t>(two_per_sm ? 2 * sms : sms, std::max<int64_t>(n_tiles, cdiv(units, kMinSlabsPerCta)));
+    const int64_t slots = nm <= 32 ? 2 * sms : sms;
+    int64_t aligned = 0;
+    for (int64_t s = 1; s <= num_k / kMinSlabsPerCta; ++s)
+      if (num_k % s == 0 && n_tiles * s <= slots) aligned = n_tiles * s;
+    if (aligned > 0 && aligned * 10 >= g * (nm <= 16 ? 8 : 7)) g = aligned;
   }
   g = std::min<int64_t>(g, units);
   return static_cast<int>(std::max<int64_t>(g, 1));
