@@ -93,6 +93,28 @@ def test_decode_partitions(decode_data, ctas):
     assert torch.equal(c1, c2)
 
 
+@pytest.mark.parametrize("name,m,ctas", [("down", 8, 96), ("down", 33, 288), ("qkv", 8, 144), ("qkv", 64, 240)])
+def test_decode_multiple_of_tiles_partitions(decode_data, name, m, ctas):
+    """CTA counts that are multiples of the tile count whose quotient does not
+    divide the tile's K slabs (112 / 3, 112 / 9, 32 / 3, 32 / 5), so ranges
+    cross tiles at shifting offsets; with 33 tokens and 64 tokens (48- and
+    64-token tiles, one CTA per SM, so more CTAs than fit at once)."""
+    import oracle as orc
+    weights, xs = decode_data
+    qw, sfw, gw, gsfw = weights[name]
+    n, k = synthetic.DECODE_SHAPES[name]
+    x = xs[k][:m].contiguous()
+    qx, sfx = orc.mx_quantize(synthetic.bits(x))
+    gx, gsfx = fp8mm.mxfp8_quantize(gu.to_dev(x))
+    ws = _workspace(m, n, k, ctas)
+    c1 = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, small_m_ctas=ctas)
+    c2 = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, small_m_ctas=ctas)
+    torch.cuda.synchronize()
+    c_ref, bound = orc.gemm_mx(qx, sfx, qw, sfw)
+    gu.check_gemm(c1, c_ref, bound, f"decode {name} m={m} ctas={ctas}")
+    assert torch.equal(c1, c2)
+
+
 @pytest.mark.parametrize("m,n,k", [(3, 200, 96), (17, 130, 4128), (64, 384, 320), (33, 1000, 64)])
 def test_decode_ragged(m, n, k):
     """Ragged shapes; the weights are quantized right before each GEMM on the
@@ -106,7 +128,7 @@ def test_decode_ragged(m, n, k):
     gx, gsfx = fp8mm.mxfp8_quantize(gu.to_dev(x))
     gw, gsfw = fp8mm.mxfp8_quantize(gu.to_dev(w))
     c_ref, bound = orc.gemm_mx(qx, sfx, qw, sfw)
-    for ctas in (0, 5):
+    for ctas in (0, 5, 10, 66):                                  # 2 tiles x 33 slabs at k = 4128
         ws = _workspace(m, n, k, ctas)
         gw, gsfw = fp8mm.mxfp8_quantize(gu.to_dev(w))          # immediately precedes the GEMM
         c = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, small_m_ctas=ctas)
