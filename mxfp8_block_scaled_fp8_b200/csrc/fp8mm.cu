@@ -418,13 +418,16 @@ static int small_m_l2_ahead(int64_t units, int64_t ctas, int64_t sms) {
 // with s dividing the tile's K slabs, so every CTA runs one segment inside
 // one tile and all contributors of a tile are equal -- when the largest such
 // count that fits the SMs (two per SM for token tiles up to 32) comes within
-// 80 % of it (16-token tiles) or 70 % (larger tiles, whose split-tile partials
+// 80 % of it (16-token tiles) or 60 % (larger tiles, whose split-tile partials
 // cost more).  Measured on B200 with back-to-back calls (GEMM alone): 6144 x
-// 4096 at m <= 32 with 192 CTAs instead of 148 is 12-17 % faster, 4096 x
-// 14336 at m <= 8 with 256 instead of 148 8 %, at m = 64 with 128 instead of
-// 148 6 %, 14336 x 4096 at m = 32 with 224 instead of 296 5 % and at m = 64
-// with 112 instead of 148 9 %; at m <= 8 there 224 is 3 % slower than 296
-// (more bytes in flight outweigh the alignment for 16-token tiles).
+// 4096 at m <= 32 with 192 CTAs instead of 148 is 12-17 % faster and at m = 64
+// with 96 instead of 148 10 %, 4096 x 14336 at m <= 8 with 256 instead of 148
+// 8 % and at m = 64 with 128 instead of 148 6 %, 14336 x 4096 at m = 32 with
+// 224 instead of 296 5 % and at m = 64 with 112 instead of 148 9 %; at m <= 8
+// there 224 is 3 % slower than 296 (more bytes in flight outweigh the
+// alignment for 16-token tiles).  Counts between the aligned ones are slower
+// than both neighbours (e.g. 6144 x 4096, m = 1: 8.5 us at 192 CTAs, 9.6-10.4
+// us at 160-240).
 constexpr int64_t kMinSlabsPerCta = 4;
 static int small_m_ctas(int64_t units, int64_t n_tiles, int64_t num_k, int nm, int64_t requested, int64_t sms) {
   int64_t g = requested;
@@ -435,7 +438,7 @@ static int small_m_ctas(int64_t units, int64_t n_tiles, int64_t num_k, int nm, i
     int64_t aligned = 0;
     for (int64_t s = 1; s <= num_k / kMinSlabsPerCta; ++s)
       if (num_k % s == 0 && n_tiles * s <= slots) aligned = n_tiles * s;
-    if (aligned > 0 && aligned * 10 >= g * (nm <= 16 ? 8 : 7)) g = aligned;
+    if (aligned > 0 && aligned * 10 >= g * (nm <= 16 ? 8 : 6)) g = aligned;
   }
   g = std::min<int64_t>(g, units);
   return static_cast<int>(std::max<int64_t>(g, 1));
