@@ -75,12 +75,16 @@ typedef struct fp8mm_opts {
   void* workspace;
   size_t workspace_bytes;
   /* Kernel choice: FP8MM_KERNEL_AUTO (small-M kernel for mxfp8_gemm with
-   * m <= 64, paired-SM tiles for m >= 256, single-SM tiles otherwise),
-   * FP8MM_KERNEL_TILED (tiled, pair or single chosen by size),
+   * m <= 64, paired-SM tiles for m >= 256, single-SM tiles otherwise, and
+   * single-SM 128x128 tiles where the 256-wide tiles would need more waves:
+   * shapes that leave most SMs idle, such as 2048 x 1024),
+   * FP8MM_KERNEL_TILED (tiled, chosen by size as for AUTO),
    * FP8MM_KERNEL_SMALL_M (weights on the MMA M side, tokens on N; mxfp8_gemm
    * only, m <= 64), FP8MM_KERNEL_TILED_1SM (persistent 128x256 tiles, one CTA
-   * per SM) or FP8MM_KERNEL_TILED_2SM (256x256 tiles on 2-CTA clusters with
-   * cta_group::2 MMAs; each CTA loads its own halves of A and B). */
+   * per SM), FP8MM_KERNEL_TILED_2SM (256x256 tiles on 2-CTA clusters with
+   * cta_group::2 MMAs; each CTA loads its own halves of A and B) or
+   * FP8MM_KERNEL_TILED_1SM_N128 (persistent 128x128 tiles, one CTA per SM,
+   * two accumulators in both scale modes). */
   int32_t kernel;
   /* Number of CTAs for the small-M kernel's stream-K split (0 = automatic:
    * one per SM, but at least 4 K slabs of 128 per CTA). */
@@ -103,6 +107,7 @@ typedef struct fp8mm_opts {
 #define FP8MM_KERNEL_SMALL_M 2
 #define FP8MM_KERNEL_TILED_1SM 3
 #define FP8MM_KERNEL_TILED_2SM 4
+#define FP8MM_KERNEL_TILED_1SM_N128 5
 
 /* ---------------------------------------------------------------- mode 1 */
 

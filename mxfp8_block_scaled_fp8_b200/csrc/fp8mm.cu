@@ -185,6 +185,8 @@ static fp8mm_status launched() {
 // ------------------------------------------------------------------ kernels' configs
 using G1 = GemmCfg<false, 256, 4, 2>;
 using G2 = GemmCfg<true, 256, 4, 1>;
+using G1n = GemmCfg<false, 128, 6, 2>;  // 128 x 128 tiles
+using G2n = GemmCfg<true, 128, 6, 2>;
 // Small-M ring depth: as many stages as shared memory holds (the weight
 // stream needs ~25 MB in flight GPU-wide to cover the loaded HBM latency).
 // Stages of the small-M kernel: token tiles up to 32 run two CTAs per SM
@@ -207,15 +209,26 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
 }
 
 // ------------------------------------------------------------------ launchers
+template <typename Cfg, typename Kern>
+static fp8mm_status launch_tiled_kernel(Kern kern, int grid, const CUtensorMap& ta, const CUtensorMap& tb,
+                                        const GemmArgs& p, cudaStream_t stream, int dev) {
+  fp8mm_status st = ensure_smem(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, dev);
+  if (st != FP8MM_OK) return st;
+  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, stream>>>(ta, tb, p);
+  return launched();
+}
+
+// Single-SM tiled kernel, 128 x 256 tiles or (n128) 128 x 128 tiles.
 // c8 != nullptr (mode 1 only): E4M3 output c8 = E4M3(C / *s_out) instead of bf16 c.
 static fp8mm_status launch_tiled(bool mx, const void* a, const void* b, const uint8_t* sfa, const uint8_t* sfb,
                                  int64_t m, int64_t n, int64_t k, const float* sa, const float* sb, void* c,
                                  int64_t ldc, cudaStream_t stream, const DeviceInfo& dev, uint8_t* c8 = nullptr,
-                                 const float* s_out = nullptr) {
+                                 const float* s_out = nullptr, bool n128 = false) {
+  const int bn = n128 ? 128 : 256;
   CUtensorMap ta, tb;
   fp8mm_status st = make_map(&ta, a, k, m, kBM);
   if (st != FP8MM_OK) return st;
-  st = make_map(&tb, b, k, n, 256);
+  st = make_map(&tb, b, k, n, bn);
   if (st != FP8MM_OK) return st;
   GemmArgs p{};
   p.m = static_cast<int>(m);
@@ -223,7 +236,7 @@ static fp8mm_status launch_tiled(bool mx, const void* a, const void* b, const ui
   p.k = static_cast<int>(k);
   p.num_k = static_cast<int>(cdiv(k, kBK));
   p.tiles_m = static_cast<int>(cdiv(m, kBM));
-  p.tiles_n = static_cast<int>(cdiv(n, 256));
+  p.tiles_n = static_cast<int>(cdiv(n, bn));
   p.num_tiles = p.tiles_m * p.tiles_n;
   p.c = static_cast<__nv_bfloat16*>(c);
   p.ldc = ldc;
@@ -237,20 +250,34 @@ static fp8mm_status launch_tiled(bool mx, const void* a, const void* b, const ui
   p.c8 = c8;
   p.s_out = s_out;
   const int grid = std::min(p.num_tiles, dev.sms);
-  if (c8 != nullptr) {
-    auto kern = gemm_tiled_kernel<false, 256, 4, 2, true>;
-    if ((st = ensure_smem(reinterpret_cast<const void*>(kern), G1::kSmemBytes, dev.device)) != FP8MM_OK) return st;
-    kern<<<grid, kGemmThreads, G1::kSmemBytes, stream>>>(ta, tb, p);
-  } else if (mx) {
-    auto kern = gemm_tiled_kernel<true, 256, 4, 1>;
-    if ((st = ensure_smem(reinterpret_cast<const void*>(kern), G2::kSmemBytes, dev.device)) != FP8MM_OK) return st;
-    kern<<<grid, kGemmThreads, G2::kSmemBytes, stream>>>(ta, tb, p);
-  } else {
-    auto kern = gemm_tiled_kernel<false, 256, 4, 2>;
-    if ((st = ensure_smem(reinterpret_cast<const void*>(kern), G1::kSmemBytes, dev.device)) != FP8MM_OK) return st;
-    kern<<<grid, kGemmThreads, G1::kSmemBytes, stream>>>(ta, tb, p);
+  if (n128) {
+    if (c8 != nullptr) return launch_tiled_kernel<G1n>(gemm_tiled_kernel<false, 128, 6, 2, true>, grid, ta, tb, p, stream, dev.device);
+    if (mx) return launch_tiled_kernel<G2n>(gemm_tiled_kernel<true, 128, 6, 2>, grid, ta, tb, p, stream, dev.device);
+    return launch_tiled_kernel<G1n>(gemm_tiled_kernel<false, 128, 6, 2>, grid, ta, tb, p, stream, dev.device);
   }
-  return launched();
+  if (c8 != nullptr) return launch_tiled_kernel<G1>(gemm_tiled_kernel<false, 256, 4, 2, true>, grid, ta, tb, p, stream, dev.device);
+  if (mx) return launch_tiled_kernel<G2>(gemm_tiled_kernel<true, 256, 4, 1>, grid, ta, tb, p, stream, dev.device);
+  return launch_tiled_kernel<G1>(gemm_tiled_kernel<false, 256, 4, 2>, grid, ta, tb, p, stream, dev.device);
+}
+
+// Tiled kernel for a call: the requested one, or (AUTO / TILED) paired-SM
+// 256 x 256 tiles from m >= 256 and single-SM 128 x 256 tiles below -- unless
+// single-SM 128 x 128 tiles need fewer waves, a 128 x 128 wave counted as
+// three quarters of a 256-wide one (half the work per SM, with relatively
+// more fixed cost: scale copies, start-up, epilogue).  That picks 128 x 128
+// where the 256-wide tiles leave most SMs idle, e.g. M 2048 x N 1024: 32
+// paired tiles on 74 SM pairs, or 128 single-SM tiles on 148 SMs.
+enum class Tiled { kPair, k1Sm, k1SmN128 };
+static Tiled tiled_kind(int kind, int64_t m, int64_t n, int64_t sms) {
+  if (kind == FP8MM_KERNEL_TILED_2SM) return Tiled::kPair;
+  if (kind == FP8MM_KERNEL_TILED_1SM) return Tiled::k1Sm;
+  if (kind == FP8MM_KERNEL_TILED_1SM_N128) return Tiled::k1SmN128;
+  const bool pair = m >= 256;
+  const int64_t big = pair ? cdiv(m, 256) * cdiv(n, 256) : cdiv(m, kBM) * cdiv(n, 256);
+  const int64_t waves_big = cdiv(big, pair ? std::max<int64_t>(1, sms / 2) : sms);
+  const int64_t waves_small = cdiv(cdiv(m, kBM) * cdiv(n, 128), sms);
+  if (3 * waves_small < 4 * waves_big) return Tiled::k1SmN128;
+  return pair ? Tiled::kPair : Tiled::k1Sm;
 }
 
 using P1 = PairCfg<false, 6, 2>;
@@ -688,16 +715,17 @@ fp8mm_status fp8_gemm(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t
   if (k > 0 && (scale_a == nullptr || scale_b == nullptr)) return FP8MM_ERR_NULL;
   if (!aligned(scale_a, 4) || !aligned(scale_b, 4)) return FP8MM_ERR_ALIGN;
   if (opt != nullptr && (opt->kernel == FP8MM_KERNEL_SMALL_M || opt->kernel < FP8MM_KERNEL_AUTO ||
-                         opt->kernel > FP8MM_KERNEL_TILED_2SM))
+                         opt->kernel > FP8MM_KERNEL_TILED_1SM_N128))
     return FP8MM_ERR_SHAPE;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != FP8MM_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (k == 0) return zero_output(c_bf16, m, n, ldc, s);
-  const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
-  const bool pair = (kind == FP8MM_KERNEL_TILED_2SM) || (kind != FP8MM_KERNEL_TILED_1SM && m >= 256);
-  if (pair) return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev);
-  return launch_tiled(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev);
+  const Tiled tk = tiled_kind(opt ? opt->kernel : FP8MM_KERNEL_AUTO, m, n, dev.sms);
+  if (tk == Tiled::kPair)
+    return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev);
+  return launch_tiled(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev,
+                      nullptr, nullptr, tk == Tiled::k1SmN128);
 }
 
 fp8mm_status fp8_gemm_e4m3_out(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t n, int64_t k,
@@ -708,7 +736,7 @@ fp8mm_status fp8_gemm_e4m3_out(const void* a_e4m3, const void* b_e4m3, int64_t m
   if (scale_out == nullptr || (k > 0 && (scale_a == nullptr || scale_b == nullptr))) return FP8MM_ERR_NULL;
   if (!aligned(scale_a, 4) || !aligned(scale_b, 4) || !aligned(scale_out, 4)) return FP8MM_ERR_ALIGN;
   if (opt != nullptr && (opt->kernel == FP8MM_KERNEL_SMALL_M || opt->kernel < FP8MM_KERNEL_AUTO ||
-                         opt->kernel > FP8MM_KERNEL_TILED_2SM))
+                         opt->kernel > FP8MM_KERNEL_TILED_1SM_N128))
     return FP8MM_ERR_SHAPE;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != FP8MM_OK) return st;
@@ -718,14 +746,13 @@ fp8mm_status fp8_gemm_e4m3_out(const void* a_e4m3, const void* b_e4m3, int64_t m
                                       static_cast<size_t>(m), s);
     return e == cudaSuccess ? FP8MM_OK : cuda_fail(e);
   }
-  const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
   auto* c8 = static_cast<uint8_t*>(c_e4m3);
-  const bool pair = (kind == FP8MM_KERNEL_TILED_2SM) || (kind != FP8MM_KERNEL_TILED_1SM && m >= 256);
-  if (pair)
+  const Tiled tk = tiled_kind(opt ? opt->kernel : FP8MM_KERNEL_AUTO, m, n, dev.sms);
+  if (tk == Tiled::kPair)
     return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, nullptr, ldc, s, dev, c8,
                        scale_out);
   return launch_tiled(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, nullptr, ldc, s, dev, c8,
-                      scale_out);
+                      scale_out, tk == Tiled::k1SmN128);
 }
 
 fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e4m3, const uint8_t* sf_b, int64_t m,
@@ -736,16 +763,17 @@ fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e
   if (!aligned(sf_a, 16) || !aligned(sf_b, 16)) return FP8MM_ERR_ALIGN;
   const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
   if (kind == FP8MM_KERNEL_SMALL_M && m > 64) return FP8MM_ERR_SHAPE;
-  if (kind < FP8MM_KERNEL_AUTO || kind > FP8MM_KERNEL_TILED_2SM) return FP8MM_ERR_SHAPE;
+  if (kind < FP8MM_KERNEL_AUTO || kind > FP8MM_KERNEL_TILED_1SM_N128) return FP8MM_ERR_SHAPE;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != FP8MM_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (k == 0) return zero_output(c_bf16, m, n, ldc, s);
   const bool small = (kind == FP8MM_KERNEL_SMALL_M) || (kind == FP8MM_KERNEL_AUTO && m <= 64);
   if (small) return launch_small_m(a_e4m3, sf_a, b_e4m3, sf_b, m, n, k, c_bf16, ldc, opt, s, dev);
-  const bool pair = (kind == FP8MM_KERNEL_TILED_2SM) || (kind != FP8MM_KERNEL_TILED_1SM && m >= 256);
-  if (pair) return launch_pair(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev);
-  return launch_tiled(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev);
+  const Tiled tk = tiled_kind(kind, m, n, dev.sms);
+  if (tk == Tiled::kPair) return launch_pair(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev);
+  return launch_tiled(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev, nullptr,
+                      nullptr, tk == Tiled::k1SmN128);
 }
 
 // Largest m whose activation is quantized inside the small-M kernel; above it

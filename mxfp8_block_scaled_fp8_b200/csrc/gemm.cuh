@@ -9,8 +9,10 @@
 //           mm_mxfp8); kind::mxf8f6f4.block_scale, scales consumed by the MMA
 //           from TMEM.
 //
-// One CTA per SM loops over 128 x kBN output tiles (grouped raster: kGroupM
-// M-tiles share each B tile while it is hot in L2).  Warp roles:
+// One CTA per SM loops over 128 x kBN output tiles, kBN = 256 or 128 (grouped
+// raster: kGroupM M-tiles share each B tile while it is hot in L2).  The
+// 128-wide tiles, with two accumulators also in mode 2, serve shapes whose
+// 256-wide tiles would leave most SMs idle.  Warp roles:
 //   warp 0      TMA producer: A/B tiles (128-byte swizzle) and, in mode 2,
 //               the 512-byte scale chunks, into a kStages-deep ring.
 //   warp 1      allocates TMEM; one lane issues tcgen05.mma (and tcgen05.cp of
@@ -291,12 +293,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------ epilogue
     // Eight warps: warp w reads TMEM sub-partition (w % 4), i.e. tile rows
     // 32*(w%4) .. +31, and one half of the tile's columns.  Each thread pulls
-    // its 128 accumulator values into registers with four loads and a single
-    // wait, then releases the accumulator at once, so the next tile's MMAs
-    // overlap the scaling, conversion and stores below.
+    // its kBN/2 accumulator values into registers with kBN/64 loads and a
+    // single wait, then releases the accumulator at once, so the next tile's
+    // MMAs overlap the scaling, conversion and stores below.
     const int sp = warp & 3;
     const int col_half = (warp - 2) >> 2;
     constexpr int kHalf = kBN / 2;
+    constexpr int kChunks = kHalf / 32;
     float s_out = 1.f, r_out = 1.f;
     bool out_fast = true;
     if constexpr (kOut8) {
@@ -304,7 +307,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       r_out = __frcp_rn(s_out);
       out_fast = quotient_fast_ok(s_out);
     }
-    static_assert(kHalf == 128, "epilogue assumes 256-column tiles");
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
@@ -314,12 +316,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sp * 32) << 16) +
                              static_cast<uint32_t>(acc * kBN + col_half * kHalf);
-      uint32_t r[4][32];
+      uint32_t r[kChunks][32];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld_32x32b_x32(t_row + ch * 32, r[ch]);
+      for (int ch = 0; ch < kChunks; ++ch) tmem_ld_32x32b_x32(t_row + ch * 32, r[ch]);
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) asm volatile("" : FP8MM_RW32(r[ch]));
+      for (int ch = 0; ch < kChunks; ++ch) asm volatile("" : FP8MM_RW32(r[ch]));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
@@ -332,7 +334,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       float s_row = 1.f;
       if constexpr (!kMX) s_row = (row < p.m) ? __ldg(p.sa + row) : 0.f;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < kChunks; ++ch) {
         const int col0 = nb * kBN + col_half * kHalf + ch * 32;
         float sbv = 1.f;
         if constexpr (!kMX) sbv = (col0 + lane < p.n) ? __ldg(p.sb + col0 + lane) : 0.f;

@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libfp8mm.so")
 
 FP8MM_OK = 0
 FP8MM_ERR_DEVICE = 7
-KERNEL_AUTO, KERNEL_TILED, KERNEL_SMALL_M, KERNEL_TILED_1SM, KERNEL_TILED_2SM = 0, 1, 2, 3, 4
+KERNEL_AUTO, KERNEL_TILED, KERNEL_SMALL_M, KERNEL_TILED_1SM, KERNEL_TILED_2SM, KERNEL_TILED_1SM_N128 = 0, 1, 2, 3, 4, 5
 
 
 class Fp8mmError(RuntimeError):

@@ -86,6 +86,13 @@ def test_argument_errors_without_a_gpu():
     assert C(P(fake), P(fake), P(fake), 2, 2, 120, 64, 1, 240, 120, 64, 0, 368, 184, None) == 3       # 120-byte rows
     assert C(P(fake + 8), P(fake), P(fake), 2, 2, 128, 64, 1, 256, 128, 64, 0, 384, 192, None) == 3   # base
     assert C(None, None, None, 0, 2, 128, 64, 1, 256, 128, 64, 0, 384, 192, None) == 0                # no tokens
+    # kernel choices: 0..5 are known, others are rejected before any device work
+    for bad in (-1, 6):
+        o = binding.Opts(None, 0, bad, 0, 0)
+        assert L.fp8_gemm(P(fake), P(fake), 4, 4, 16, P(fake), P(fake), P(fake), 8, ctypes.byref(o), None) == 2
+        assert L.mxfp8_gemm(P(fake), P(fake), P(fake), P(fake), 4, 4, 32, P(fake), 8, ctypes.byref(o), None) == 2
+        assert E(P(fake), P(fake), 4, 4, 16, P(fake), P(fake), P(fake), P(fake), 8, ctypes.byref(o), None) == 2
+    assert binding.KERNEL_TILED_1SM_N128 == 5
     # empty problems are no-ops and need no device
     assert L.fp8_gemm(None, None, 0, 4, 16, None, None, None, 8, None, None) == 0
     assert L.mxfp8_quantize(None, 0, 64, 64, None, 64, None, None) == 0

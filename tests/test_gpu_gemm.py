@@ -76,13 +76,15 @@ def test_tiny_rowwise_full():
     run_rowwise(a, bt, label="tiny 128x256x512")
 
 
-@pytest.mark.parametrize("kernel", [fp8mm.KERNEL_TILED_2SM, fp8mm.KERNEL_TILED_1SM], ids=["2sm", "1sm"])
+@pytest.mark.parametrize("kernel", [fp8mm.KERNEL_AUTO, fp8mm.KERNEL_TILED_2SM, fp8mm.KERNEL_TILED_1SM,
+                                    fp8mm.KERNEL_TILED_1SM_N128], ids=["auto", "2sm", "1sm", "1sm_n128"])
 def test_qk_mx_full(kernel):
     a, bt = synthetic.qk()
     run_mx(a, bt, label="qk 2048x1024x4096", kernel=kernel)
 
 
-@pytest.mark.parametrize("kernel", [fp8mm.KERNEL_AUTO, fp8mm.KERNEL_TILED_1SM], ids=["auto", "1sm"])
+@pytest.mark.parametrize("kernel", [fp8mm.KERNEL_AUTO, fp8mm.KERNEL_TILED_1SM, fp8mm.KERNEL_TILED_1SM_N128],
+                         ids=["auto", "1sm", "1sm_n128"])
 def test_attn_rowwise_sampled(kernel):
     a, bt = synthetic.attn()
     run_rowwise(a, bt, sample=_rows_cols(8192, 2048, 192, 64, 2), label="attn 8192x2048x8192", kernel=kernel)
@@ -106,7 +108,8 @@ def test_mx_tall_raster_groups_ragged():
 
 # ------------------------------------------------------------ shapes and edges
 
-KERNELS = pytest.mark.parametrize("kernel", [fp8mm.KERNEL_TILED_1SM, fp8mm.KERNEL_TILED_2SM], ids=["1sm", "2sm"])
+KERNELS = pytest.mark.parametrize("kernel", [fp8mm.KERNEL_TILED_1SM, fp8mm.KERNEL_TILED_2SM, fp8mm.KERNEL_TILED_1SM_N128],
+                                  ids=["1sm", "2sm", "1sm_n128"])
 
 
 @KERNELS

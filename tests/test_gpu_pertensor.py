@@ -100,7 +100,8 @@ def _check_e4m3_gemm(c_codes, c_ref, bound, s_out, label):
                            f"got {got[bad[:3]]}, interval [{dec[lo][bad[:3]]}, {dec[hi][bad[:3]]}]")
 
 
-@pytest.mark.parametrize("kernel", [fp8mm.KERNEL_AUTO, fp8mm.KERNEL_TILED_1SM, fp8mm.KERNEL_TILED_2SM])
+@pytest.mark.parametrize("kernel", [fp8mm.KERNEL_AUTO, fp8mm.KERNEL_TILED_1SM, fp8mm.KERNEL_TILED_2SM,
+                                    fp8mm.KERNEL_TILED_1SM_N128])
 def test_e4m3_out_tiny_and_ragged(kernel):
     import oracle as orc
     for (m, n, k) in [(128, 256, 512), (300, 130, 96), (257, 513, 1040)]:
