@@ -66,12 +66,18 @@ typedef int fp8mm_status;
 
 /* Optional knobs of the GEMM calls (pass NULL for defaults). */
 typedef struct fp8mm_opts {
-  /* Device scratch for the small-M split-K kernel: fp32 partial tiles plus one
-   * 32-bit arrival counter per output tile.  Caller-owned.  It must be zeroed
-   * once before first use (e.g. cudaMemsetAsync); every successful call leaves
-   * the counters zero again.  After a call that reported FP8MM_ERR_DEVICE it
-   * must be zeroed again.  Calls sharing one workspace must not overlap on
-   * the GPU.  NULL disables split-K. */
+  /* Device scratch for split K: fp32 partial tiles plus 32-bit arrival
+   * counters, fp8mm_workspace_bytes(m, n, k, small_m_ctas) bytes, 256-byte
+   * aligned.  Used by the small-M kernel (mxfp8_gemm, m <= 64) and, for
+   * m > 64, by the paired-SM kernel where its 256 x 256 tiles fill less than
+   * one wave of SM pairs (the K range of each tile is then split over several
+   * pairs; fp8mm_workspace_bytes is 0 for shapes that are not split).
+   * Caller-owned.  It must be zeroed once before first use (e.g.
+   * cudaMemsetAsync); every successful call leaves the counters zero again.
+   * After a call that reported FP8MM_ERR_DEVICE it must be zeroed again.
+   * Calls sharing one workspace must not overlap on the GPU.  NULL disables
+   * split K.  A workspace too small for the split the shape takes is
+   * FP8MM_ERR_WORKSPACE. */
   void* workspace;
   size_t workspace_bytes;
   /* Kernel choice: FP8MM_KERNEL_AUTO (small-M kernel for mxfp8_gemm with
@@ -133,7 +139,9 @@ fp8mm_status fp8_quantize_rowwise(const void* x_bf16, int64_t rows, int64_t k, i
  *   scale_a [m] fp32, scale_b [n] fp32, c [m, n] bf16 with row stride ldc.
  * Requires k % 16 == 0, a/b 16-byte aligned, c 2-byte aligned, ldc >= n (rows
  * whose address is 16-byte aligned are written with 16-byte stores).
- * m == 0 or n == 0 is a no-op; k == 0 writes zeros.  opt may be NULL. */
+ * m == 0 or n == 0 is a no-op; k == 0 writes zeros.  opt may be NULL; with
+ * opt->workspace, m > 64 shapes that fill less than one wave of SM pairs split
+ * K over the pairs (see fp8mm_opts.workspace). */
 fp8mm_status fp8_gemm(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t n, int64_t k,
                       const float* scale_a, const float* scale_b, void* c_bf16, int64_t ldc,
                       const fp8mm_opts* opt, void* stream);
@@ -214,7 +222,9 @@ fp8mm_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
  * With m <= 64 the small-M (decode) kernel runs: weights b fill the MMA's
  * 128-row side, tokens the N side, and K is split stream-K style over the SMs
  * when opt->workspace is given (see fp8mm_workspace_bytes); partial sums are
- * reduced deterministically (fixed order) by the last CTA of each tile. */
+ * reduced deterministically (fixed order) by the last CTA of each tile.  With
+ * m > 64 and a workspace, shapes whose 256 x 256 tiles fill less than one
+ * wave of SM pairs split each tile's K range over pairs the same way. */
 fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e4m3, const uint8_t* sf_b,
                         int64_t m, int64_t n, int64_t k, void* c_bf16, int64_t ldc, const fp8mm_opts* opt,
                         void* stream);
@@ -245,8 +255,10 @@ fp8mm_status mxfp8_quantize_gemm(const void* a_bf16, int64_t lda, const void* b_
  * (each 256-byte aligned).  0 for m outside [1, 64]. */
 size_t fp8mm_quantize_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas);
 
-/* Workspace bytes the small-M kernel needs for this shape with `ctas` CTAs
- * (0 = one per SM of the current device; on a host without a GPU, 148). */
+/* Workspace bytes a GEMM of this shape uses: for m <= 64 those of the
+ * small-M kernel with `ctas` CTAs (0 = its automatic choice); for m > 64 those
+ * of the paired-SM kernel's K split (`ctas` ignored), 0 when the shape is not
+ * split.  The current device's SM count decides; on a host without a GPU, 148. */
 size_t fp8mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas);
 
 /* ---------------------------------------------------------------- KV cache */

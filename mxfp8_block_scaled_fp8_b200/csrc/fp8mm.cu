@@ -249,6 +249,7 @@ static fp8mm_status launch_tiled(bool mx, const void* a, const void* b, const ui
   p.timeout_ns = wait_timeout_ns();
   p.c8 = c8;
   p.s_out = s_out;
+  p.split = 1;
   const int grid = std::min(p.num_tiles, dev.sms);
   if (n128) {
     if (c8 != nullptr) return launch_tiled_kernel<G1n>(gemm_tiled_kernel<false, 128, 6, 2, true>, grid, ta, tb, p, stream, dev.device);
@@ -326,10 +327,50 @@ static fp8mm_status max_pairs(const void* kern, int smem, int threads, const Dev
 // 8192 x 2048 x 8192 (B 16 MB, L2-resident) 16 are 1.6 % slower than 8.
 static int pair_group_m(int64_t n, int64_t k) { return n * k > (int64_t{64} << 20) ? 2 * kPairGroupM : kPairGroupM; }
 
+// K parts per tile of the paired-SM kernel (split K): where its 256 x 256
+// tiles fill less than one wave of SM pairs and K has at least 64 slabs of
+// 128, the most parts that still fit in one wave, each of at least 16 slabs,
+// at most 8; else 1.  Only for m > 64 (below that mxfp8_gemm runs the
+// small-M kernel).  The fp32 partials cost a write and a read of 256 KB per
+// part and tile through L2, so short K gains nothing: measured on B200,
+// 512 x 2048 x 8192 (16 tiles, 4 parts of 16 slabs) takes 23.2 us against
+// 29.5 us unsplit (MX), but 2048 x 1024 x 4096 with 2 parts of 16 slabs 21.4
+// us against 18.3 us on 128 x 128 single-SM tiles.
+static int pair_split(int64_t m, int64_t n, int64_t k, int64_t sms) {
+  const int64_t num_k = cdiv(k, kBK);
+  if (m <= 64 || num_k < 64) return 1;
+  const int64_t tiles = cdiv(m, 256) * cdiv(n, 256);
+  const int64_t pairs = std::max<int64_t>(1, sms / 2);
+  const int64_t s = std::min<int64_t>(std::min<int64_t>(pairs / tiles, num_k / 16), 8);
+  return static_cast<int>(std::max<int64_t>(1, s));
+}
+static size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+// Workspace of a split-K paired launch: the partials, then the counters.
+static size_t pair_partials_bytes(int64_t m, int64_t n, int split) {
+  return round256(static_cast<size_t>(cdiv(m, 256) * cdiv(n, 256)) * split * 2 * kPairPartFloats * sizeof(float));
+}
+static size_t pair_split_bytes(int64_t m, int64_t n, int split) {
+  if (split <= 1) return 0;
+  return pair_partials_bytes(m, n, split) + round256(static_cast<size_t>(cdiv(m, 256) * cdiv(n, 256)) * 2 * 4);
+}
+// Split for a tiled call: > 1 when a workspace is given, the kernel choice
+// allows the paired kernel (AUTO, TILED, TILED_2SM) and the shape is split;
+// -1 when that workspace is too small or misaligned.
+static int tiled_split(const fp8mm_opts* opt, int kind, int64_t m, int64_t n, int64_t k, int64_t sms) {
+  if (opt == nullptr || opt->workspace == nullptr) return 1;
+  if (kind != FP8MM_KERNEL_AUTO && kind != FP8MM_KERNEL_TILED && kind != FP8MM_KERNEL_TILED_2SM) return 1;
+  const int s = pair_split(m, n, k, sms);
+  if (s <= 1) return 1;
+  if (opt->workspace_bytes < pair_split_bytes(m, n, s) || !aligned(opt->workspace, 256)) return -1;
+  return s;
+}
+
+// split > 1: K split into that many parts per tile, partials and counters in
+// the workspace (pair_split_bytes(m, n, split) bytes, counters zero).
 static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uint8_t* sfa, const uint8_t* sfb,
                                 int64_t m, int64_t n, int64_t k, const float* sa, const float* sb, void* c,
                                 int64_t ldc, cudaStream_t stream, const DeviceInfo& dev, uint8_t* c8 = nullptr,
-                                const float* s_out = nullptr) {
+                                const float* s_out = nullptr, int split = 1, void* workspace = nullptr) {
   CUtensorMap ta, tb, tsa, tsb;
   fp8mm_status st = make_map(&ta, a, k, m, 128);
   if (st != FP8MM_OK) return st;
@@ -361,6 +402,11 @@ static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uin
   p.c8 = c8;
   p.s_out = s_out;
   p.group_m = pair_group_m(n, k);
+  p.split = split > 1 ? split : 1;
+  if (p.split > 1) {
+    p.partials = static_cast<float*>(workspace);
+    p.tickets = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + pair_partials_bytes(m, n, p.split));
+  }
   const void* kern = mx ? reinterpret_cast<const void*>(gemm_pair_kernel<true, 6, 1>)
                      : c8 ? reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2, true>)
                           : reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2>);
@@ -369,7 +415,7 @@ static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uin
   if ((st = ensure_smem(kern, smem, dev.device)) != FP8MM_OK) return st;
   int pairs = 0;
   if ((st = max_pairs(kern, smem, threads, dev, &pairs)) != FP8MM_OK) return st;
-  pairs = std::min(pairs, p.num_tiles);
+  pairs = std::min(pairs, p.num_tiles * p.split);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -578,16 +624,14 @@ fp8mm_status fp8mm_sf_from_canonical(const uint8_t* canonical, int64_t rows, int
 }
 
 size_t fp8mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas) {
-  if (m <= 0 || n <= 0 || k <= 0 || m > 64) return 0;
-  int g = ctas;
-  if (g <= 0) {
-    int dev = 0, sms = 0;
-    g = (cudaGetDevice(&dev) == cudaSuccess &&
-         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
-            ? sms
-            : 148;
-    cudaGetLastError();  // a host without a GPU leaves an error behind
-  }
+  if (m <= 0 || n <= 0 || k <= 0) return 0;
+  int dev = 0, sms = 0;
+  if (!(cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0))
+    sms = 148;
+  cudaGetLastError();  // a host without a GPU leaves an error behind
+  if (m > 64) return pair_split_bytes(m, n, pair_split(m, n, k, sms));
+  int g = ctas > 0 ? ctas : sms;
   const int64_t units = cdiv(n, 128) * cdiv(k, 128);
   g = small_m_ctas(units, cdiv(n, 128), cdiv(k, 128), small_m_tile(m), ctas, g);
   const size_t tickets = static_cast<size_t>(cdiv(n, 128)) * sizeof(unsigned);
@@ -721,7 +765,13 @@ fp8mm_status fp8_gemm(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t
   if ((st = current_device(&dev)) != FP8MM_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (k == 0) return zero_output(c_bf16, m, n, ldc, s);
-  const Tiled tk = tiled_kind(opt ? opt->kernel : FP8MM_KERNEL_AUTO, m, n, dev.sms);
+  const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
+  const int split = tiled_split(opt, kind, m, n, k, dev.sms);
+  if (split < 0) return FP8MM_ERR_WORKSPACE;
+  if (split > 1)
+    return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev,
+                       nullptr, nullptr, split, opt->workspace);
+  const Tiled tk = tiled_kind(kind, m, n, dev.sms);
   if (tk == Tiled::kPair)
     return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev);
   return launch_tiled(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev,
@@ -747,7 +797,13 @@ fp8mm_status fp8_gemm_e4m3_out(const void* a_e4m3, const void* b_e4m3, int64_t m
     return e == cudaSuccess ? FP8MM_OK : cuda_fail(e);
   }
   auto* c8 = static_cast<uint8_t*>(c_e4m3);
-  const Tiled tk = tiled_kind(opt ? opt->kernel : FP8MM_KERNEL_AUTO, m, n, dev.sms);
+  const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
+  const int split = tiled_split(opt, kind, m, n, k, dev.sms);
+  if (split < 0) return FP8MM_ERR_WORKSPACE;
+  if (split > 1)
+    return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, nullptr, ldc, s, dev, c8,
+                       scale_out, split, opt->workspace);
+  const Tiled tk = tiled_kind(kind, m, n, dev.sms);
   if (tk == Tiled::kPair)
     return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, nullptr, ldc, s, dev, c8,
                        scale_out);
@@ -770,6 +826,11 @@ fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e
   if (k == 0) return zero_output(c_bf16, m, n, ldc, s);
   const bool small = (kind == FP8MM_KERNEL_SMALL_M) || (kind == FP8MM_KERNEL_AUTO && m <= 64);
   if (small) return launch_small_m(a_e4m3, sf_a, b_e4m3, sf_b, m, n, k, c_bf16, ldc, opt, s, dev);
+  const int split = tiled_split(opt, kind, m, n, k, dev.sms);
+  if (split < 0) return FP8MM_ERR_WORKSPACE;
+  if (split > 1)
+    return launch_pair(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev, nullptr,
+                       nullptr, split, opt->workspace);
   const Tiled tk = tiled_kind(kind, m, n, dev.sms);
   if (tk == Tiled::kPair) return launch_pair(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev);
   return launch_tiled(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev, nullptr,

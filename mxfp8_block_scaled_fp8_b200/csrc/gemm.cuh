@@ -54,6 +54,9 @@ struct GemmArgs {
   int sfb_row_tiles;         // ceil(n / 128): 128-row tiles present in sfb
   uint64_t timeout_ns;
   int group_m;               // paired-SM kernel: 256-row tiles per raster group
+  int split;                 // paired-SM kernel: K parts per tile (1 = whole K, no partials)
+  float* partials;           // split > 1: fp32 partials [num_tiles * split][2][128 * 256]
+  unsigned* tickets;         // split > 1: arrivals per (tile, CTA rank), zero between calls
 };
 
 // Epilogue store of one thread's 32 consecutive outputs v[0..31] of row `row`

@@ -28,6 +28,15 @@
 // MMA issuer; warps 2..17 epilogue (four per TMEM sub-partition, 64
 // accumulator columns each, drained into registers with one wait so the
 // accumulator is free again at once).
+//
+// Split K (split > 1, for shapes whose tiles fill less than one wave of SM
+// pairs): the work units are (tile, K part) with part j covering K slabs
+// [floor(j*num_k/split), floor((j+1)*num_k/split)); pairs take units in turn.
+// Each CTA stores its fp32 partial (its 128 rows x 256 columns) in the
+// workspace, bumps the (tile, rank) arrival counter, and the last to arrive
+// sums the parts in part order (fixed, so the result does not depend on
+// timing), applies the scales, writes C and resets the counter.  No CTA waits
+// for another.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -54,8 +63,8 @@ struct PairCfg {
   static constexpr int kOffSfa = kOffB + kStages * kBBytes;
   static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
   static constexpr int kOffBar = kOffSfb + kStages * kSfbBytes;
-  // full, empty per stage; acc_full, acc_empty per accumulator; drain
-  static constexpr int kNumBars = 2 * kStages + 2 * kAccStages + 1;
+  // full, empty per stage; acc_full, acc_empty per accumulator; drain; epi_sync
+  static constexpr int kNumBars = 2 * kStages + 2 * kAccStages + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   // bytes of both CTAs' loads, all completing on the leader's barrier
@@ -78,6 +87,19 @@ __device__ __forceinline__ void pair_tile_coords(int t, const GemmArgs& p, int& 
   nb = r / gm;
 }
 
+// Work unit u: tile t and its K slabs [kb0, kb1).
+__device__ __forceinline__ void pair_unit(int u, const GemmArgs& p, int& t, int& kb0, int& kb1) {
+  t = u / p.split;
+  const int j = u - t * p.split;
+  kb0 = static_cast<int>(static_cast<int64_t>(j) * p.num_k / p.split);
+  kb1 = static_cast<int>(static_cast<int64_t>(j + 1) * p.num_k / p.split);
+}
+
+// Floats of one CTA's partial tile: 16 epilogue warps x 2 chunks x 32
+// columns x 32 lanes (= 128 rows x 256 columns), stored so that each warp's
+// 32 lanes write 128 contiguous bytes per column.
+constexpr int kPairPartFloats = 16 * 2 * 32 * 32;
+
 // GemmArgs fields as in gemm.cuh, with tiles_m = ceil(m/256), tiles_n =
 // ceil(n/256).  tmSFA: 3-D map over the scale layout viewed as uint32
 // [n_rt][n_kc][128]; tmSFB: 4-D map [n_rt][4 replicas, stride 0][n_kc][128]
@@ -95,8 +117,11 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + kAccStages;
   uint64_t* drain = acc_empty + kAccStages;
+  uint64_t* epi_sync = drain + 1;  // the 16 epilogue warps meet here (split K; bounded)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 8);
+  const int num_units = p.num_tiles * p.split;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -115,6 +140,7 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
       mbar_init(&acc_empty[a], 32);  // 16 epilogue warps in each CTA of the pair
     }
     mbar_init(drain, 1);
+    mbar_init(epi_sync, 16);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -141,10 +167,11 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
       int stage = 0;
       uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
       bool ok = true;
-      for (int t = pair; ok && t < p.num_tiles; t += npairs) {
-        int mb, nb;
+      for (int u = pair; ok && u < num_units; u += npairs) {
+        int t, kb0, kb1, mb, nb;
+        pair_unit(u, p, t, kb0, kb1);
         pair_tile_coords(t, p, mb, nb);
-        for (int kb = 0; kb < p.num_k; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) {
             ok = false;
             break;
@@ -187,11 +214,13 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int t = pair; ok && t < p.num_tiles; t += npairs) {
+      for (int u = pair; ok && u < num_units; u += npairs) {
+        int t, kb0, kb1;
+        pair_unit(u, p, t, kb0, kb1);
         if (!mbar_wait_cluster(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, kSiteMmaAccEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
-        for (int kb = 0; kb < p.num_k; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_cluster(&full[stage], phase, p.timeout_ns, abort_flag, kSiteMmaFull)) {
             ok = false;
             break;
@@ -207,11 +236,11 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
 #pragma unroll
             for (int kk = 0; kk < kBK / kMmaK; ++kk)
               mma_mxf8f6f4_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8f6f4(256, 256, kk, kk), sfa_t,
-                                sfa_t + 8u, (kb | kk) != 0);
+                                sfa_t + 8u, kb != kb0 || kk != 0);
           } else {
 #pragma unroll
             for (int kk = 0; kk < kBK / kMmaK; ++kk)
-              mma_f8f6f4_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_f8f6f4(256, 256), (kb | kk) != 0);
+              mma_f8f6f4_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_f8f6f4(256, 256), kb != kb0 || kk != 0);
           }
           tc_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == kStages) {
@@ -242,9 +271,19 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
       out_fast = quotient_fast_ok(s_out);
     }
     int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int t = pair; t < p.num_tiles; t += npairs) {
-      int mb, nb;
+    uint32_t acc_phase = 0, sync_phase = 0;
+    const int wl = warp - Cfg::kEpiWarp0;  // 0..15
+    // The 16 epilogue warps meet (split K); false if the wait expired or the CTA aborted.
+    auto epi_meet = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_sync);
+      const bool ok = mbar_wait(epi_sync, sync_phase, p.timeout_ns, abort_flag, kSiteEpiSync);
+      sync_phase ^= 1u;
+      return ok;
+    };
+    for (int u = pair; u < num_units; u += npairs) {
+      int t, kb0, kb1, mb, nb;
+      pair_unit(u, p, t, kb0, kb1);
       pair_tile_coords(t, p, mb, nb);
       if (!mbar_wait_cluster(&acc_full[acc], acc_phase, p.timeout_ns, abort_flag, kSiteEpiAccFull)) break;
       tc_fence_after();
@@ -267,6 +306,49 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
       const int row = mb * 256 + static_cast<int>(rank) * 128 + sp * 32 + lane;
       float s_row = 1.f;
       if constexpr (!kMX) s_row = (row < p.m) ? __ldg(p.sa + row) : 0.f;
+      if (p.split > 1) {
+        // Publish this part, count it; the last part to arrive reduces.
+        float* mine = p.partials + (static_cast<int64_t>(u) * 2 + rank) * kPairPartFloats + wl * 2048 + lane;
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) mine[ch * 1024 + j * 32] = __uint_as_float(r[ch][j]);
+        // The 16 warps' partial stores are ordered before one thread's
+        // acquire-release counter increment at GPU scope (the barrier between
+        // them is CTA-scope release/acquire and release is cumulative); the
+        // last part's increment acquires every earlier part's stores, and the
+        // barrier after it hands them to its other threads.
+        if (!epi_meet()) break;
+        unsigned* ticket = p.tickets + static_cast<int64_t>(t) * 2 + rank;
+        if (threadIdx.x == Cfg::kEpiWarp0 * 32) {
+          unsigned prev;
+          asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ticket) : "memory");
+          *last_flag = (prev == static_cast<unsigned>(p.split - 1)) ? 1 : 0;
+        }
+        if (!epi_meet()) break;
+        if (*last_flag == 0) continue;
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const int col0 = nb * 256 + quarter * 64 + ch * 32;
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          for (int part = 0; part < p.split; ++part) {
+            const float* src = p.partials + (static_cast<int64_t>(t * p.split + part) * 2 + rank) * kPairPartFloats +
+                               wl * 2048 + ch * 1024 + lane;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += __ldcg(src + j * 32);
+          }
+          if constexpr (!kMX) {
+            const float sbv = (col0 + lane < p.n) ? __ldg(p.sb + col0 + lane) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = v[j] * s_row * __shfl_sync(0xFFFFFFFFu, sbv, j);
+          }
+          store_out32<kOut8>(p, row, col0, v, s_out, r_out, out_fast);
+        }
+        if (threadIdx.x == Cfg::kEpiWarp0 * 32) *ticket = 0u;
+        continue;
+      }
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         const int col0 = nb * 256 + quarter * 64 + ch * 32;

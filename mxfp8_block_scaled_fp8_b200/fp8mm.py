@@ -127,9 +127,18 @@ def fp8_quantize_rowwise(x: torch.Tensor, q: torch.Tensor | None = None, scale: 
     return q, scale
 
 
+def _ws_opts(workspace, kernel, small_m_ctas=0, flags=0):
+    return Opts(workspace.data_ptr() if workspace is not None else None,
+                workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                kernel, small_m_ctas, flags)
+
+
 def fp8_gemm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
-             c: torch.Tensor | None = None, kernel: int = KERNEL_AUTO, stream=None) -> torch.Tensor:
-    """C bf16 [m, n] = diag(scale_a) (A x B^T) diag(scale_b); a [m,k], b [n,k] E4M3 codes."""
+             c: torch.Tensor | None = None, kernel: int = KERNEL_AUTO, stream=None,
+             workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """C bf16 [m, n] = diag(scale_a) (A x B^T) diag(scale_b); a [m,k], b [n,k] E4M3 codes.
+    workspace (zeroed once, workspace_bytes(m, n, k) bytes): lets m > 64 shapes that fill less than one
+    wave of SM pairs split K over the pairs."""
     a, b = _u8(a), _u8(b)
     _need(a, torch.uint8, "a"); _need(b, torch.uint8, "b")
     _need(scale_a, torch.float32, "scale_a"); _need(scale_b, torch.float32, "scale_b")
@@ -139,7 +148,7 @@ def fp8_gemm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: t
         raise ValueError("a [m,k] and b [n,k] must be contiguous with the same k")
     if c is None:
         c = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
-    opts = Opts(None, 0, kernel, 0, 0)
+    opts = _ws_opts(workspace, kernel)
     _check("fp8_gemm", lib().fp8_gemm(a.data_ptr(), b.data_ptr(), m, n, k, scale_a.data_ptr(), scale_b.data_ptr(),
                                       c.data_ptr(), _ld(c, "c"), ctypes.byref(opts), _stream(stream)))
     return c
@@ -173,8 +182,8 @@ def fp8_quantize_static(x: torch.Tensor, scale: torch.Tensor, q: torch.Tensor | 
 
 def fp8_gemm_e4m3_out(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
                       scale_out: torch.Tensor, c: torch.Tensor | None = None, kernel: int = KERNEL_AUTO,
-                      stream=None) -> torch.Tensor:
-    """E4M3 codes uint8 [m, n] of diag(scale_a) (A x B^T) diag(scale_b) / scale_out."""
+                      stream=None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """E4M3 codes uint8 [m, n] of diag(scale_a) (A x B^T) diag(scale_b) / scale_out (workspace as fp8_gemm)."""
     a, b = _u8(a), _u8(b)
     _need(a, torch.uint8, "a"); _need(b, torch.uint8, "b")
     _need(scale_a, torch.float32, "scale_a"); _need(scale_b, torch.float32, "scale_b")
@@ -186,7 +195,7 @@ def fp8_gemm_e4m3_out(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, s
     if c is None:
         c = torch.empty((m, n), dtype=torch.uint8, device=a.device)
     c = _u8(c)
-    opts = Opts(None, 0, kernel, 0, 0)
+    opts = _ws_opts(workspace, kernel)
     _check("fp8_gemm_e4m3_out", lib().fp8_gemm_e4m3_out(
         a.data_ptr(), b.data_ptr(), m, n, k, scale_a.data_ptr(), scale_b.data_ptr(), scale_out.data_ptr(),
         c.data_ptr(), _ld(c, "c"), ctypes.byref(opts), _stream(stream)))
@@ -245,6 +254,8 @@ def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch
                c: torch.Tensor | None = None, workspace: torch.Tensor | None = None, kernel: int = KERNEL_AUTO,
                small_m_ctas: int = 0, weights_ready: bool = False, stream=None) -> torch.Tensor:
     """C bf16 [m, n] = block-scaled A x B^T; a [m,k], b [n,k] codes with their library-layout scales.
+    workspace (zeroed once, workspace_bytes(m, n, k, small_m_ctas) bytes): the small-M kernel's stream-K
+    split for m <= 64; for m > 64 the K split of shapes that fill less than one wave of SM pairs.
     weights_ready: b and sf_b were complete before the preceding kernel on the stream started (see
     FP8MM_FLAG_WEIGHTS_READY)."""
     a, b = _u8(a), _u8(b)
@@ -256,9 +267,7 @@ def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch
         raise ValueError("a [m,k] and b [n,k] must be contiguous with the same k")
     if c is None:
         c = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
-    opts = Opts(workspace.data_ptr() if workspace is not None else None,
-                workspace.numel() * workspace.element_size() if workspace is not None else 0,
-                kernel, small_m_ctas, FLAG_WEIGHTS_READY if weights_ready else 0)
+    opts = _ws_opts(workspace, kernel, small_m_ctas, FLAG_WEIGHTS_READY if weights_ready else 0)
     _check("mxfp8_gemm", lib().mxfp8_gemm(a.data_ptr(), sf_a.data_ptr(), b.data_ptr(), sf_b.data_ptr(), m, n, k,
                                           c.data_ptr(), _ld(c, "c"), ctypes.byref(opts), _stream(stream)))
     return c

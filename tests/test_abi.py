@@ -103,7 +103,17 @@ def test_workspace_sizes():
     # 2 * G * 128 * NM floats (256-byte aligned) + one counter per 128-row tile
     assert fp8mm.workspace_bytes(64, 14336, 4096, 148) == 2 * 148 * 128 * 64 * 4 + 512
     assert fp8mm.workspace_bytes(1, 4096, 14336, 148) == 2 * 148 * 128 * 16 * 4 + 256
-    assert fp8mm.workspace_bytes(65, 4096, 4096, 148) == 0            # only for m <= 64
+    # m > 64: the paired kernel's K split, on a host without a GPU for 148 SMs (74 pairs);
+    # partials of 128 x 256 fp32 per (tile, part, CTA rank), then 2 counters per tile (256-byte rounded)
+    part = 128 * 256 * 4
+    assert fp8mm.workspace_bytes(65, 4096, 8192, 148) == 16 * 4 * 2 * part + 256     # 16 tiles, 4 parts
+    assert fp8mm.workspace_bytes(512, 2048, 8192) == 16 * 4 * 2 * part + 256         # the same tiles
+    assert fp8mm.workspace_bytes(2048, 512, 16384) == 16 * 4 * 2 * part + 256        # 128 slabs: 74 // 16 = 4
+    assert fp8mm.workspace_bytes(1024, 1024, 8192) == 16 * 4 * 2 * part + 256
+    assert fp8mm.workspace_bytes(2048, 1024, 8192) == 32 * 2 * 2 * part + 256        # 32 tiles, 2 parts
+    assert fp8mm.workspace_bytes(2048, 1024, 4096) == 0                              # 32 K slabs: no split
+    assert fp8mm.workspace_bytes(65, 4096, 4096) == 0
+    assert fp8mm.workspace_bytes(8192, 22016, 8192) == 0                             # more tiles than pairs
     assert fp8mm.workspace_bytes(8, 128, 128, 148) == 2 * 1 * 128 * 16 * 4 + 256   # clamped to 1 unit
     # activation-quantizing GEMM: the same for m <= 8, plus the quantized activation and scales above
     assert fp8mm.quantize_gemm_workspace_bytes(8, 14336, 4096, 148) == fp8mm.workspace_bytes(8, 14336, 4096, 148)

@@ -106,6 +106,74 @@ def test_mx_tall_raster_groups_ragged():
     run_mx(a, bt, sample=(rows, cols), label=f"mx {m}x{n}x{k}")
 
 
+# ------------------------------------------------------------ split K (paired kernel, m > 64)
+
+def _ws(m, n, k):
+    nbytes = fp8mm.workspace_bytes(m, n, k)
+    assert nbytes > 0, "shape expected to split"
+    return torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+
+
+@pytest.mark.parametrize("mode", ["mx", "rowwise"])
+@pytest.mark.parametrize("m,n,k", [(512, 2048, 8192),       # 16 tiles, 4 parts of 16 K slabs
+                                   (2048, 1024, 8192),      # 32 tiles, 2 parts of 32
+                                   (65, 4096, 8192),        # 16 tiles of which most rows are padding
+                                   (300, 600, 8960)])       # 6 tiles; 70 K slabs in 4 parts: 17, 18, 17, 18
+def test_split_k_full(mode, m, n, k):
+    """Shapes whose 256 x 256 tiles fill less than one wave of SM pairs split
+    K over the pairs when a workspace is given; the full result meets the bar,
+    a second call with the same workspace is bit-identical (the counters are
+    back at zero) and equals no split within the bar."""
+    a = synthetic.random_bf16((m, k), seed=m + 7)
+    bt = synthetic.random_bf16((n, k), seed=n + 8, sigma=0.05)
+    ws = _ws(m, n, k)
+    import oracle as orc
+    if mode == "mx":
+        qa, sfa = orc.mx_quantize(synthetic.bits(a))
+        qb, sfb = orc.mx_quantize(synthetic.bits(bt))
+        ga, gsfa = fp8mm.mxfp8_quantize(gu.to_dev(a))
+        gb, gsfb = fp8mm.mxfp8_quantize(gu.to_dev(bt))
+        call = lambda: fp8mm.mxfp8_gemm(ga, gsfa, gb, gsfb, workspace=ws)
+        c_ref, bound = orc.gemm_mx(qa, sfa, qb, sfb)
+    else:
+        qa, sa = orc.quantize_rowwise(synthetic.bits(a))
+        qb, sb = orc.quantize_rowwise(synthetic.bits(bt))
+        ga, gsa = fp8mm.fp8_quantize_rowwise(gu.to_dev(a))
+        gb, gsb = fp8mm.fp8_quantize_rowwise(gu.to_dev(bt))
+        call = lambda: fp8mm.fp8_gemm(ga, gb, gsa, gsb, workspace=ws)
+        c_ref, bound = orc.gemm_rowwise(qa, qb, sa, sb)
+    c1 = call()
+    c2 = call()
+    torch.cuda.synchronize()
+    gu.check_gemm(c1, c_ref, bound, f"split-K {mode} {m}x{n}x{k}")
+    assert torch.equal(c1, c2)
+    assert not ws[-256:].any()                               # the arrival counters are back at zero
+    assert fp8mm.last_device_error() == 0
+
+
+def test_split_k_e4m3_out_and_errors():
+    import oracle as orc
+    m, n, k = 512, 2048, 8192
+    a = synthetic.random_bf16((m, k), seed=61)
+    bt = synthetic.random_bf16((n, k), seed=62)
+    ga, gsa = fp8mm.fp8_quantize_rowwise(gu.to_dev(a))
+    gb, gsb = fp8mm.fp8_quantize_rowwise(gu.to_dev(bt))
+    so = torch.tensor([0.5], dtype=torch.float32, device="cuda")
+    ws = _ws(m, n, k)
+    c_split = fp8mm.fp8_gemm_e4m3_out(ga, gb, gsa, gsb, so, workspace=ws)
+    c_plain = fp8mm.fp8_gemm_e4m3_out(ga, gb, gsa, gsb, so)
+    torch.cuda.synchronize()
+    dec = orc.e4m3_decode_table()
+    x, y = dec[c_split.cpu().numpy()], dec[c_plain.cpu().numpy()]
+    # same accumulator up to summation order: codes equal or adjacent
+    lo = np.minimum(x, y); hi = np.maximum(x, y)
+    codes = np.sort(np.unique(dec[np.isfinite(dec)]))
+    idx_lo, idx_hi = np.searchsorted(codes, lo), np.searchsorted(codes, hi)
+    assert np.all(idx_hi - idx_lo <= 1)
+    with pytest.raises(fp8mm.Fp8mmError):
+        fp8mm.fp8_gemm(ga, gb, gsa, gsb, workspace=torch.zeros(1024, dtype=torch.uint8, device="cuda"))
+
+
 # ------------------------------------------------------------ shapes and edges
 
 KERNELS = pytest.mark.parametrize("kernel", [fp8mm.KERNEL_TILED_1SM, fp8mm.KERNEL_TILED_2SM, fp8mm.KERNEL_TILED_1SM_N128],
