@@ -6,7 +6,7 @@
 // the m tokens the N side (padded to kNM = 16..64), so D = B_tile x A^T lands
 // in TMEM as 128 weight rows x kNM tokens.  At these sizes the call is bound
 // by streaming the weight bytes from HBM, so the K range of the n/128 weight
-// tiles is split stream-K style over (up to) one CTA per SM: CTA b owns units
+// tiles is split stream-K style over up to two CTAs per SM: CTA b owns units
 // [b*U/G, (b+1)*U/G) of the U = n_tiles * num_k (tile, 128-wide K slab)
 // units.  A tile covered by one CTA is written directly; otherwise each
 // contributor stores its fp32 partial in the workspace, bumps the tile's
