@@ -62,8 +62,10 @@ struct GemmArgs {
 // Epilogue store of one thread's 32 consecutive outputs v[0..31] of row `row`
 // from column col0: bf16 round-to-nearest-even into p.c, or with kOut8 the
 // E4M3 codes of v / s_out (quotient_sat, IEEE division when !fast) into p.c8.
-// Full 32-column runs whose address is 16-byte aligned use 16-byte stores;
-// ragged or unaligned runs store element by element.
+// Full 32-column runs store 32 bytes at a time where the address is 32-byte
+// aligned (bf16: each store fills a whole 32-byte sector), else 16 bytes at a
+// time where it is 16-byte aligned; ragged or unaligned runs store element by
+// element.
 template <bool kOut8>
 __device__ __forceinline__ void store_out32(const GemmArgs& p, int row, int col0, const float (&v)[32], float s_out,
                                             float r_out, bool fast) {
@@ -95,7 +97,11 @@ __device__ __forceinline__ void store_out32(const GemmArgs& p, int row, int col0
       packed[j] = *reinterpret_cast<uint32_t*>(&h);
     }
     __nv_bfloat16* dst = p.c + static_cast<int64_t>(row) * p.ldc + col0;
-    if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+    if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
+      st_global_v8(dst, packed[0], packed[1], packed[2], packed[3], packed[4], packed[5], packed[6], packed[7]);
+      st_global_v8(dst + 16, packed[8], packed[9], packed[10], packed[11], packed[12], packed[13], packed[14],
+                   packed[15]);
+    } else if (col0 + 32 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4)
         *reinterpret_cast<uint4*>(dst + q4 * 8) =

@@ -124,6 +124,13 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// 32-byte global store (sm_100 256-bit vector store); dst 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* dst, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                             uint32_t w4, uint32_t w5, uint32_t w6, uint32_t w7) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w0), "r"(w1), "r"(w2),
+               "r"(w3), "r"(w4), "r"(w5), "r"(w6), "r"(w7)
+               : "memory");
+}
 // Prefetches into L2 (no destination, no completion to wait for): a 2-D
 // tile of a tensor map (x aligned as for tma_load_2d), and an untiled range
 // (16-byte aligned address, size a multiple of 16).
