@@ -317,7 +317,6 @@ static fp8mm_status max_pairs(const void* kern, int smem, int threads, const Dev
   return FP8MM_OK;
 }
 
-// c8 != nullptr (mode 1 only): E4M3 output c8 = E4M3(C / *s_out) instead of bf16 c.
 // 256-row output tiles per raster group of the paired-SM kernel.  Within a
 // group the tiles run down M, then across N, so B is read from DRAM once per
 // group and the group's A rows are reused from L2.  Where B is too large to
@@ -365,8 +364,10 @@ static int tiled_split(const fp8mm_opts* opt, int kind, int64_t m, int64_t n, in
   return s;
 }
 
-// split > 1: K split into that many parts per tile, partials and counters in
-// the workspace (pair_split_bytes(m, n, split) bytes, counters zero).
+// Paired-SM kernel.  c8 != nullptr (mode 1 only): E4M3 output c8 =
+// E4M3(C / *s_out) instead of bf16 c.  split > 1: K split into that many parts
+// per tile, partials and counters in the workspace (pair_split_bytes(m, n,
+// split) bytes, counters zero).
 static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uint8_t* sfa, const uint8_t* sfb,
                                 int64_t m, int64_t n, int64_t k, const float* sa, const float* sb, void* c,
                                 int64_t ldc, cudaStream_t stream, const DeviceInfo& dev, uint8_t* c8 = nullptr,
