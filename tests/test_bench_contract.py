@@ -1,0 +1,40 @@
+"""bench.py's measurement plumbing, on the CPU: the ncu traffic figure is
+reported only for the kernel sources it was captured on, the rotated operand
+copies of the per-row measurements exceed L2, and the reference arm prints the
+contract's JSON line."""
+import json
+import os
+import subprocess
+import sys
+
+import bench
+
+
+def test_traffic_only_for_the_captured_sources(monkeypatch):
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        entry = json.load(f)["mxfp8_gemm_ffn_up"]
+    monkeypatch.setattr(bench, "_src_hash", lambda: entry["src_hash"])
+    assert bench._ncu_traffic("mxfp8_gemm_ffn_up") == entry["bytes_per_launch"]
+    monkeypatch.setattr(bench, "_src_hash", lambda: "0" * 16)      # the kernels changed since the capture
+    assert bench._ncu_traffic("mxfp8_gemm_ffn_up") is None
+    assert bench._ncu_traffic("no_such_kernel") is None
+
+
+def test_rotated_copies_exceed_l2():
+    for nbytes in (1 << 20, 58_720_256, 180 << 20, 400 << 20):
+        n = bench._copies(nbytes)
+        assert n >= 2 and n * nbytes >= 320 << 20                 # > the 126 MB L2 in total
+
+
+def test_reference_arm_json_line():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "1"],
+                       cwd=bench.ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "impl", "cpu_baseline", "e2e", "config"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["higher_is_better"] is True
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
