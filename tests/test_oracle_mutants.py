@@ -14,6 +14,7 @@ import oracle
 from tests import test_oracle_formats as F
 from tests import test_oracle_gemm as G
 from tests import test_oracle_quant as Q
+from tests import test_oracle_quotient as D
 from tests import test_oracle_static_concat as S
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
@@ -35,6 +36,10 @@ MUTANTS = {
                      "double prod = g->dec[a[t]] * g->dec[g->qb[(t * g->n + j) % (g->n * g->k)]];"),
     "mx_block_index_dropped": ("(int)g->sfb[j * nkb + blk] - 254", "(int)g->sfb[j * nkb] - 254"),
     "subnormal_decode_wrong": ("mag = ldexp((double)m, -9);", "mag = ldexp((double)m, -10);"),
+    "rowwise_reciprocal_multiply": ("float v = bf16_to_float(xr[j]) / s;",
+                                    "float v = bf16_to_float(xr[j]) * (1.0f / s);"),
+    "static_reciprocal_multiply": ("float v = bf16_to_float(c->x[r * c->ld_x + j]) / c->s;",
+                                   "float v = bf16_to_float(c->x[r * c->ld_x + j]) * (1.0f / c->s);"),
 }
 
 PINS = [
@@ -49,6 +54,8 @@ PINS = [
     lambda o: S.test_tensor_scale_closed_forms(3),
     lambda o: S.test_static_with_power_of_two_scale_is_exact_scaling(-1),
     lambda o: S.test_static_with_the_row_scale_is_the_row_quantizer(),
+    D.test_rowwise_quotient_is_ieee_division_at_ties, D.test_rowwise_quotient_is_ieee_division_many_scales,
+    D.test_static_quotient_is_ieee_division,
 ]
 
 
