@@ -59,6 +59,19 @@ struct GemmArgs {
   unsigned* tickets;         // split > 1: arrivals per (tile, CTA rank), zero between calls
 };
 
+// Per-token / per-channel scaling of an fp32 accumulator, sa * sb * acc
+// (page "从 DeepGEMM 到 vLLM", listing 1: scale_a[m] and scale_b[n]).  The
+// scale product is rounded once and applied where it is a normal fp32; where
+// it is not (a subnormal row or column scale, or sa * sb past the fp32 range)
+// the accumulator is scaled by each in turn, so that neither a huge row scale
+// meeting a tiny column scale overflows on the way nor a subnormal product
+// loses its significand.
+__device__ __forceinline__ float scale_acc(float acc, float sa, float sb) {
+  const float sab = sa * sb;
+  const float m = fabsf(sab);
+  return (m >= 0x1p-126f && m <= 0x1.fffffep127f) ? acc * sab : (acc * sa) * sb;
+}
+
 // Epilogue store of one thread's 32 consecutive outputs v[0..31] of row `row`
 // from column col0: bf16 round-to-nearest-even into p.c, or with kOut8 the
 // E4M3 codes of v / s_out (quotient_sat, IEEE division when !fast) into p.c8.
@@ -351,7 +364,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           v[j] = __uint_as_float(r[ch][j]);
-          if constexpr (!kMX) v[j] = v[j] * s_row * __shfl_sync(0xFFFFFFFFu, sbv, j);
+          if constexpr (!kMX) v[j] = scale_acc(v[j], s_row, __shfl_sync(0xFFFFFFFFu, sbv, j));
         }
         store_out32<kOut8>(p, row, col0, v, s_out, r_out, out_fast);
       }

@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
           if constexpr (!kMX) {
             const float sbv = (col0 + lane < p.n) ? __ldg(p.sb + col0 + lane) : 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = v[j] * s_row * __shfl_sync(0xFFFFFFFFu, sbv, j);
+            for (int j = 0; j < 32; ++j) v[j] = scale_acc(v[j], s_row, __shfl_sync(0xFFFFFFFFu, sbv, j));
           }
           store_out32<kOut8>(p, row, col0, v, s_out, r_out, out_fast);
         }
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           v[j] = __uint_as_float(r[ch][j]);
-          if constexpr (!kMX) v[j] = v[j] * s_row * __shfl_sync(0xFFFFFFFFu, sbv, j);
+          if constexpr (!kMX) v[j] = scale_acc(v[j], s_row, __shfl_sync(0xFFFFFFFFu, sbv, j));
         }
         store_out32<kOut8>(p, row, col0, v, s_out, r_out, out_fast);
       }

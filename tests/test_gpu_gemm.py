@@ -257,3 +257,79 @@ def test_repeat_calls_bit_identical():
     torch.cuda.synchronize()
     assert torch.equal(c1, c2)
     assert fp8mm.last_device_error() == 0
+
+
+# ------------------------------------------------------------ the method's edge values
+
+def _edge_operands(m, n, k):
+    """A and B^T with the cases the two scale rules single out: all-zero rows and
+    32-element blocks (MX exponent 127, row scale 1), rows small enough that
+    every MX exponent is clamped to 0 (the padding scale) and the row scale is
+    an fp32 subnormal, blocks whose maximum is exactly 448 times a power of
+    two (mapped to 448 itself), rows scaled by 1e25 and 1e-30, and a row of
+    +-bf16 max."""
+    a = synthetic.random_bf16((m, k), seed=71, sigma=2.0)
+    bt = synthetic.random_bf16((n, k), seed=72, sigma=1.0)
+    bmax = torch.finfo(torch.bfloat16).max
+    a[0] = 0.0
+    a[1, 32:64] = 0.0
+    a[2] *= 2e-37                                   # MX: every block at the low clamp
+    a[3, 64:96] = 448.0 * 2 ** -5                   # amax-exact blocks
+    a[3, 96:128] = -448.0 * 2 ** 9
+    a[4] *= 1e25
+    a[5] *= 1e-30
+    a[6] = bmax
+    a[6, 1::2] = -bmax
+    a[m - 1, :k // 2] = 0.0
+    bt[0] = 0.0
+    bt[1, :32] = 0.0
+    bt[2] *= 1e-36
+    bt[3, 32:64] = 448.0 * 2 ** -12
+    bt[n - 1] *= 1e4
+    return a, bt
+
+
+def _check_edge(c, c_ref, bound, label):
+    """The bar on every element whose exact value lies inside the range bf16
+    (and the fp32 accumulator) can hold: products of the +-bf16 max row pass
+    it, and tiny-times-tiny products (below 1e-30) fall under it -- there the
+    only representable answers are +-inf and (nearly) zero."""
+    inside = (bound > 1e-30) & (bound < 1e37)
+    assert inside.sum() >= c.numel() - 3 * c.shape[1] - 2 * c.shape[0]
+    mask = torch.from_numpy(inside).cuda()
+    gu.check_gemm(c[mask], c_ref[inside], bound[inside], label)
+    tiny = torch.from_numpy(bound <= 1e-30).cuda()
+    assert torch.all(c[tiny].float().abs() <= 1e-30), f"{label}: underflowing products not near zero"
+
+
+@KERNELS
+@pytest.mark.parametrize("mode", ["mx", "rowwise"])
+def test_edge_values_tiled(mode, kernel):
+    import oracle as orc
+    m, n, k = 300, 520, 1024
+    a, bt = _edge_operands(m, n, k)
+    if mode == "mx":
+        qa, sfa = orc.mx_quantize(synthetic.bits(a))
+        qb, sfb = orc.mx_quantize(synthetic.bits(bt))
+        assert sfa[2].max() == 0 and sfa[0].min() == 127      # the clamp and the zero rule are exercised
+        ga, gsfa = fp8mm.mxfp8_quantize(gu.to_dev(a))
+        gb, gsfb = fp8mm.mxfp8_quantize(gu.to_dev(bt))
+        c = fp8mm.mxfp8_gemm(ga, gsfa, gb, gsfb, kernel=kernel)
+        c_ref, bound = orc.gemm_mx(qa, sfa, qb, sfb)
+    else:
+        qa, sa = orc.quantize_rowwise(synthetic.bits(a))
+        qb, sb = orc.quantize_rowwise(synthetic.bits(bt))
+        ga, gsa = fp8mm.fp8_quantize_rowwise(gu.to_dev(a))
+        gb, gsb = fp8mm.fp8_quantize_rowwise(gu.to_dev(bt))
+        c = fp8mm.fp8_gemm(ga, gb, gsa, gsb, kernel=kernel)
+        c_ref, bound = orc.gemm_rowwise(qa, qb, sa, sb)
+    torch.cuda.synchronize()
+    _check_edge(c, c_ref, bound, f"edge values {mode} kernel {kernel}")
+    assert torch.all(c[0] == 0)                                 # zero row
+    assert fp8mm.last_device_error() == 0
+
+
+def test_attn_rowwise_full():
+    """The attention-shaped per-token GEMM 8192 x 2048 x 8192 in full."""
+    a, bt = synthetic.attn()
+    run_rowwise(a, bt, label="attn 8192x2048x8192 full")
