@@ -140,6 +140,15 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
+def percentiles(xs):
+    """p10 / p50 / p90 of a list of per-step times (nearest rank)."""
+    v = sorted(xs)
+    if not v:
+        return None
+    pick = lambda q: v[min(len(v) - 1, max(0, int(round(q * (len(v) - 1)))))]
+    return {"p10": pick(0.10), "p50": pick(0.50), "p90": pick(0.90), "mean": sum(v) / len(v)}
+
+
 def job_tflops(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
     """Whole-job throughput: every rank runs `steps` steps of its own replica."""
     return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
@@ -336,6 +345,74 @@ def _rows_measurements(fp8mm, synthetic, peaks, only=None):
     return out
 
 
+def _sustained(step, gemm, stream, local, pci, seconds: float = 3.0, k: int = 100):
+    """The headline step back to back for `seconds` (the GPU settles at its
+    power cap); then k more steps and k GEMM calls, each timed alone with CUDA
+    events, with the clocks sampled meanwhile."""
+    import torch
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < seconds:
+        for _ in range(50):
+            step()
+        torch.cuda.synchronize()
+        n += 50
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def timed(f):
+        out = []
+        for _ in range(k):
+            ev[0].record(stream)
+            f()
+            ev[1].record(stream)
+            ev[1].synchronize()
+            out.append(ev[0].elapsed_time(ev[1]))
+        return out
+
+    with ClockSampler(local, pci_bus_id=pci) as clocks:
+        s_list = timed(step)
+        g_list = timed(gemm)
+    st, gm = percentiles(s_list), percentiles(g_list)
+    return {"warm_seconds": seconds, "warm_steps": n, "calls_timed": k, "step_ms": st, "gemm_ms": gm["p50"],
+            "gemm_ms_pct": gm, "TFLOPS_per_step": FLOPS_PER_STEP / (st["p50"] * 1e-3) / 1e12,
+            "clocks": clocks.summary(),
+            "note": "after several seconds of back-to-back steps (power cap); each call timed alone, median"}
+
+
+def _yardstick(torch, dev):
+    """torch._scaled_mm (cuBLASLt FP8) on the same GPU in the same run: a
+    library yardstick, not a target and not the roofline denominator."""
+    out = {"what": "torch._scaled_mm e4m3 x e4m3 -> bf16, best of 10 calls after 3 warm-up calls; "
+                   "a library yardstick, not a target"}
+    try:
+        shapes = {"8192x8192x8192_per_tensor": (8192, 8192, 8192, False),
+                  "8192x22016x8192_rowwise": (8192, 22016, 8192, True),
+                  "8192x2048x8192_rowwise": (8192, 2048, 8192, True)}
+        for name, (m, n, k, rowwise) in shapes.items():
+            a = torch.randn((m, k), device=dev).to(torch.float8_e4m3fn)
+            b = torch.randn((n, k), device=dev).to(torch.float8_e4m3fn)
+            sa = torch.ones((m, 1) if rowwise else (), device=dev)
+            sb = torch.ones((1, n) if rowwise else (), device=dev)
+            f = lambda: torch._scaled_mm(a, b.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
+            for _ in range(3):
+                f()
+            torch.cuda.synchronize()
+            best = None
+            for _ in range(10):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                f()
+                e1.record()
+                e1.synchronize()
+                t = e0.elapsed_time(e1)
+                best = t if best is None else min(best, t)
+            out[name] = {"ms": best, "TFLOPS": 2.0 * m * n * k / (best * 1e-3) / 1e12}
+            del a, b
+    except Exception as e:  # a library limitation is reported, not fatal
+        out["error"] = f"{type(e).__name__}: {e}"[:200]
+    return out
+
+
 # ---------------------------------------------------------------- our arm
 
 def run_ours(args):
@@ -394,8 +471,11 @@ def run_ours(args):
     if ws > 1:
         dist.barrier()
     total_ms = t_start.elapsed_time(t_end)
-    q_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in evs) / args.steps
-    g_ms = sum(e1.elapsed_time(e2) for _, e1, e2 in evs) / args.steps
+    q_list = [e0.elapsed_time(e1) for e0, e1, _ in evs]
+    g_list = [e1.elapsed_time(e2) for _, e1, e2 in evs]
+    s_list = [e0.elapsed_time(e2) for e0, _, e2 in evs]
+    q_ms = sum(q_list) / args.steps
+    g_ms = sum(g_list) / args.steps
     total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
     value = job_tflops(FLOPS_PER_STEP, args.steps, ws, total_ms)
@@ -448,6 +528,13 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e2e_ms, dev)
     del x_devs, c_devs
 
+    # the same step back to back for a few seconds: the GPU settles at its
+    # power cap, where the short timed region above runs at burst clocks
+    sustained = None
+    if not args.no_sustained:
+        sustained = _sustained(step, lambda: fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c), stream, local, pci)
+    yard = _yardstick(torch, dev) if (rank == 0 and not args.no_rows) else None
+
     rows = None
     if rank == 0 and not args.no_rows:
         rows = _rows_measurements(fp8mm, synthetic, peaks, args.only)
@@ -468,6 +555,9 @@ def run_ours(args):
                 "pipelining": "H2D, kernels and D2H on three streams with two device buffer sets"},
         "gpu_launches": 2 * args.steps,
         "kernels": {"mxfp8_quantize_ms": q_ms, "mxfp8_gemm_ms": g_ms},
+        "per_step_ms": {"step": percentiles(s_list), "mxfp8_quantize": percentiles(q_list),
+                        "mxfp8_gemm": percentiles(g_list),
+                        "note": "CUDA events around each call of every timed step (nearest-rank percentiles)"},
         "roofline": {"bound": "tensor", "kernel": "gemm_pair_kernel<mx> (mxfp8_gemm, 256x256 tiles on 2-CTA clusters)", "achieved": achieved,
                      "peak": fp8_peak, "unit": "TFLOP/s", "frac": achieved / fp8_peak,
                      "traffic": _ncu_traffic("mxfp8_gemm_ffn_up"),
@@ -482,8 +572,17 @@ def run_ours(args):
                               "traffic": _ncu_traffic("mxfp8_quantize_x")},
         "clocks": clocks.summary(),
     }
+    if sustained is not None:
+        sustained["gemm_frac_of_burst_peak"] = FLOPS_PER_STEP / (sustained["gemm_ms"] * 1e-3) / 1e12 / fp8_peak
+        sustained["gemm_frac_of_sustained_peak"] = (FLOPS_PER_STEP / (sustained["gemm_ms"] * 1e-3) / 1e12
+                                                    / (2.0 * peaks["bf16_tflops_sustained"]))
+        line["sustained"] = sustained
+    if yard is not None:
+        line["yardstick"] = yard
     if rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(CPU_SAMPLE_ROWS, _oracle_workload(x_cpu, w_cpu))
+        if not args.no_rows:
+            line["cpu_baseline"]["per_config"] = cpu_per_config()
     if rows is not None:
         line["rows"] = rows
     if rank == 0:
@@ -518,6 +617,57 @@ def cpu_baseline(rows: int, prepared=None):
             "kind": "oracle", "seconds": dt,
             "sample": f"{rows} of {M} rows of the ffn_up step (mx-quantize those rows of X, then their full "
                       f"rows of C against all {N} columns, fp64 exact accumulation); W quantized beforehand"}
+
+
+def cpu_per_config(gemm_sample_rows: int = 16):
+    """The oracle timed on every configuration shape: the quantizer of each
+    mode on every operand (rowwise for the per-token configurations, MX for
+    the block-scaled ones; decode weights once, each activation per case), the
+    GEMM in full for tiny, qk and every decode case, and on `gemm_sample_rows`
+    full rows of C for attn and ffn_up (their full GEMMs take minutes)."""
+    import oracle
+    from mxfp8_block_scaled_fp8_b200 import synthetic as S
+    out = {}
+
+    def timed(name, f, units, unit, **extra):
+        t = time.perf_counter()
+        r = f()
+        dt = time.perf_counter() - t
+        out[name] = {"seconds": dt, unit: units / dt / 1e6 if unit == "Melem/s" else units / dt / 1e9, **extra}
+        return r
+
+    def rowwise_case(name, a, bt, sample):
+        qa, sa = timed(f"{name}.quantize_rowwise_A", lambda: oracle.quantize_rowwise(S.bits(a)), a.numel(), "Melem/s")
+        qb, sb = timed(f"{name}.quantize_rowwise_B", lambda: oracle.quantize_rowwise(S.bits(bt)), bt.numel(), "Melem/s")
+        r = qa.shape[0] if sample is None else sample
+        timed(f"{name}.gemm", lambda: oracle.gemm_rowwise(qa[:r], qb, sa[:r], sb, want_bound=False),
+              r * qb.shape[0] * qa.shape[1], "GMAC/s", rows=f"{r} of {qa.shape[0]}")
+
+    def mx_case(name, a, bt, sample):
+        qa, sfa = timed(f"{name}.mx_quantize_A", lambda: oracle.mx_quantize(S.bits(a)), a.numel(), "Melem/s")
+        qb, sfb = timed(f"{name}.mx_quantize_B", lambda: oracle.mx_quantize(S.bits(bt)), bt.numel(), "Melem/s")
+        r = qa.shape[0] if sample is None else sample
+        timed(f"{name}.gemm", lambda: oracle.gemm_mx(qa[:r], sfa[:r], qb, sfb, want_bound=False),
+              r * qb.shape[0] * qa.shape[1], "GMAC/s", rows=f"{r} of {qa.shape[0]}")
+
+    rowwise_case("tiny", *S.tiny(), None)
+    mx_case("qk", *S.qk(), None)
+    rowwise_case("attn", *S.attn(), gemm_sample_rows)
+    mx_case("ffn_up", *S.ffn_up(), gemm_sample_rows)
+    ws_, xs = S.decode()
+    for name, w in ws_.items():
+        n, k = S.DECODE_SHAPES[name]
+        qw, sfw = timed(f"decode.{name}.mx_quantize_W", lambda: oracle.mx_quantize(S.bits(w)), w.numel(), "Melem/s")
+        for m in S.DECODE_M:
+            x = xs[k][:m]
+            qx, sfx = timed(f"decode.{name}_m{m}.mx_quantize_X", lambda: oracle.mx_quantize(S.bits(x)), x.numel(),
+                            "Melem/s")
+            timed(f"decode.{name}_m{m}.gemm", lambda: oracle.gemm_mx(qx, sfx, qw, sfw, want_bound=False),
+                  m * n * k, "GMAC/s", rows=f"{m} of {m}")
+    out["_about"] = ("CPU oracle (plain C, fp64 exact accumulation) on the host cores; the same seeded bf16 inputs "
+                     "as the GPU rows; 'rows' gives how much of C was computed")
+    out["_cores"] = oracle.default_threads()
+    return out
 
 
 def run_reference(args):
@@ -560,6 +710,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-sustained", action="store_true", help="skip the sustained (power-cap) loop")
     ap.add_argument("--only", default=None, help="regex: measure only the matching per-row cases")
     ap.add_argument("--rows-only", action="store_true", help="skip the headline step (profiling of single rows)")
     args = ap.parse_args()

@@ -38,3 +38,12 @@ def test_reference_arm_json_line():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_percentiles_nearest_rank():
+    p = bench.percentiles([float(i) for i in range(1, 102)])      # 1 .. 101
+    assert (p["p10"], p["p50"], p["p90"]) == (11.0, 51.0, 91.0)
+    assert p["mean"] == 51.0
+    assert bench.percentiles([]) is None
+    q = bench.percentiles([3.0])
+    assert q["p10"] == q["p50"] == q["p90"] == 3.0
