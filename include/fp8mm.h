@@ -107,6 +107,12 @@ typedef struct fp8mm_opts {
  * sf_b were complete before the preceding kernel started (e.g. weights
  * quantized at load time); never when the preceding kernel writes them. */
 #define FP8MM_FLAG_WEIGHTS_READY 1u
+/* The small-M kernel reduces a split whose CTA count is tile-aligned (s CTAs
+ * per 128-row weight tile, 2 <= s <= 8, s dividing ceil(k / 128)) inside
+ * thread-block clusters of s CTAs, through distributed shared memory, and
+ * then needs no workspace.  With this flag it reduces such splits through
+ * the workspace instead (identical results; for comparison and testing). */
+#define FP8MM_FLAG_SPLIT_VIA_WORKSPACE 2u
 
 #define FP8MM_KERNEL_AUTO 0
 #define FP8MM_KERNEL_TILED 1
@@ -319,7 +325,8 @@ int fp8mm_version(void);
  *   mxfp8_gemm.  Requires 1 <= m <= 64 (else FP8MM_ERR_SHAPE), k % 32 == 0,
  *   and at most 16384 weight tiles, i.e. n <= 2097152 (else
  *   FP8MM_ERR_WORKSPACE: the request does not fit the fixed scratch).  The
- *   stream-K split uses as many CTAs as the scratch holds, up to one per SM.
+ *   stream-K split uses the CTA count mxfp8_gemm would choose, capped at what
+ *   the scratch holds (508 CTAs for up to 16 tokens, 127 for 49..64).
  *
  * Allocates nothing: no cudaMalloc / cudaFree and no allocating library
  * call.  The first call on each device looks up the scratch array's device

@@ -14,6 +14,17 @@
 // (a fixed order, so results do not depend on timing), writes bf16 and
 // resets the counter.  No CTA ever waits for another.
 //
+// With kCR (cluster reduction) the CTA count is tile-aligned: s = G / n_tiles
+// CTAs per weight tile, s dividing the tile's K slabs, so CTA b runs the one
+// segment b % s of tile b / s, and the s contributors of a tile are launched
+// as one thread-block cluster.  Each writes its fp32 partial into its own
+// (idle) weight ring, signals every peer's mbarrier, and then sums the slice
+// of weight rows [r*128/s, (r+1)*128/s) that its rank r owns over all s
+// partials, read through distributed shared memory in rank order (the same
+// order as the workspace reduction, so the two give identical bits).  No
+// workspace and no global round trip; the cluster meets once more before
+// exit so that no CTA leaves while a peer may still read its shared memory.
+//
 // With kQX (m <= 8) the activation arrives as bf16 and is quantized inside
 // the kernel (the per-call activation quantization of page "[sglang]
 // FlashInfer v0.6.7 MXFP8 Gemm 통합", section 2, fused into the GEMM): two
@@ -58,6 +69,7 @@ struct DecodeArgs {
   int l2_ahead;        // slabs past the staged ones whose weights are prefetched into L2 at the start
   const __nv_bfloat16* x;  // kQX: bf16 activation [m, k]
   int64_t ldx;             // kQX: its row stride in elements
+  int cluster_s;           // kCR: CTAs per weight tile (= the cluster size)
 };
 
 template <int kNM, int kStages, bool kQX = false>
@@ -79,14 +91,16 @@ struct DecodeCfg {
   static constexpr int kOffSfw = kOffX + kStages * kXBytes;
   static constexpr int kOffSfx = kOffSfw + kStages * 512;
   static constexpr int kOffBar = kOffSfx + kStages * 512;
-  // full, empty per stage; acc_full, acc_empty x2; drain; epi_sync
-  static constexpr int kNumBars = 2 * kStages + 2 * 2 + 2;
+  // full, empty per stage; acc_full, acc_empty x2; drain; epi_sync; red_ready (kCR)
+  static constexpr int kNumBars = 2 * kStages + 2 * 2 + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static constexpr int kSfCol0 = 2 * kNM;
   static constexpr int kColsUsed = kSfCol0 + 8 * kStages;
   static constexpr int kTmemCols = kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128 : kColsUsed <= 256 ? 256 : 512;
   static_assert(kSmemBytes * kMinBlocksPerSm + 1024 * (kMinBlocksPerSm - 1) <= 232448, "shared memory budget");
+  // kCR: a CTA's fp32 partial tile [kNM][128] lives in its weight ring
+  static_assert(kNM * 128 * 4 <= kStages * kWBytes, "partial tile fits the weight ring");
 };
 
 __device__ __forceinline__ int64_t dec_unit_start(int b, const DecodeArgs& p) {
@@ -112,9 +126,76 @@ __device__ __forceinline__ void regs_fence_16(uint32_t* r) {
                  "+r"(r[15]));
 }
 
+__device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+
+// Cluster reduction of split tile t (kCR): the CTA of rank `rank` sums weight
+// rows [4 q0, 4 q1) -- its share of the tile's 32 row quads -- over the S
+// partials red[token][row] of the cluster's CTAs, in rank order, and writes
+// the m tokens' bf16 outputs.  tid is 0..127 (the four epilogue warps).  All
+// of a thread's distributed-shared-memory loads (ITEMS x S 16-byte vectors)
+// are issued before the first sum, so the reduction costs about one remote
+// round trip.  S = 3 stands for every split this kernel is not specialised
+// for (the loop bounds then use the runtime count).
+template <int S, int kNM>
+__device__ __forceinline__ void cluster_reduce_slice(const float* red, int rank, int t, int tid, const DecodeArgs& p) {
+  const int s = (S == 3) ? p.cluster_s : S;
+  constexpr int kMaxQuads = (S == 3) ? 11 : (32 + S - 1) / S;   // S == 3: any s in 3..6
+  constexpr int kItems = (kMaxQuads * kNM + 127) / 128;
+  constexpr int kSrc = (S == 3) ? 6 : S;
+  // specialised splits hold every load of the thread at once (<= 84 floats);
+  // the generic one item at a time
+  constexpr int kBatch = (S == 3) ? 1 : kItems;
+  const int q0 = rank * 32 / s, nq = (rank + 1) * 32 / s - q0;
+  const int total = nq * p.m;
+  const uint32_t base = smem_u32(red);
+#pragma unroll
+  for (int it0 = 0; it0 < kItems; it0 += kBatch) {
+    float4 v[kBatch][kSrc];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int idx = tid + (it0 + b) * 128;
+      const int j = idx / nq;
+      const uint32_t a = base + static_cast<uint32_t>((j * 128 + (q0 + idx - j * nq) * 4) * 4);
+#pragma unroll
+      for (int q = 0; q < kSrc; ++q)
+        v[b][q] = (idx < total && q < s) ? ld_shared_cluster_v4(mapa_shared(a, static_cast<uint32_t>(q)))
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int idx = tid + (it0 + b) * 128;
+      if (idx >= total) continue;
+      const int j = idx / nq;
+      const int quad = q0 + (idx - j * nq);
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < kSrc; ++q) {
+        if (q >= s) break;
+        sum.x += v[b][q].x;
+        sum.y += v[b][q].y;
+        sum.z += v[b][q].z;
+        sum.w += v[b][q].w;
+      }
+      const float o[4] = {sum.x, sum.y, sum.z, sum.w};
+      const int n0 = t * 128 + quad * 4;
+      __nv_bfloat16* dst = p.c + static_cast<int64_t>(j) * p.ldc + n0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (n0 + e < p.n) dst[e] = __float2bfloat16_rn(o[e]);
+    }
+  }
+}
+
 // tmX: the quantized activation (E4M3 [m, k], 128-byte swizzle, box 128 x
 // kNM); unused with kQX (the activation comes as p.x).
-template <int kNM, int kStages, bool kQX>
+template <int kNM, int kStages, bool kQX, bool kCR = false>
 __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
                                   DecodeCfg<kNM, kStages, kQX>::kMinBlocksPerSm)
     gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -128,6 +209,7 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint64_t* epi_sync = drain + 1;  // the four epilogue warps meet here (bounded)
+  uint64_t* red_ready = epi_sync + 1;  // kCR: every peer's four epilogue warps have written their partial
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 8);
@@ -151,6 +233,7 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
     }
     mbar_init(drain, 1);
     mbar_init(epi_sync, 4);
+    if (kCR) mbar_init(red_ready, 4 * p.cluster_s);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -163,7 +246,10 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kCR)
+    cluster_sync_all();  // every peer's red_ready is initialised before anyone can arrive on it
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -291,6 +377,49 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
       mbar_wait(drain, 0, p.timeout_ns, nullptr, kSiteDrain);
     }
     __syncwarp();
+  } else if (kCR && warp < Cfg::kQuantWarp0) {
+    // ------------------------------------------------------ epilogue, cluster reduction
+    griddep_wait();  // C may still be in use by the preceding kernel
+    const int sp = warp & 3;
+    const int nl = sp * 32 + lane;  // weight row inside the tile
+    const int ns = p.cluster_s;
+    const int rank = static_cast<int>(cluster_ctarank());
+    bool ok = mbar_wait(&acc_full[0], 0, p.timeout_ns, abort_flag, kSiteEpiAccFull);
+    uint32_t r[kNM];
+#pragma unroll
+    for (int j = 0; j < kNM; ++j) r[j] = 0u;
+    if (ok) {
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(sp * 32) << 16);
+#pragma unroll
+      for (int ch = 0; ch < kNM / 16; ++ch) tmem_ld_32x32b_x16(t_row + ch * 16, r + ch * 16);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int ch = 0; ch < kNM / 16; ++ch) regs_fence_16(r + ch * 16);
+    }
+    // The weight ring is idle: every TMA write into it was consumed by an MMA
+    // that completed before acc_full.  Partial [token j][row] as fp32.
+    float* red = reinterpret_cast<float*>(smem + Cfg::kOffW);
+    fence_proxy_async_smem();
+#pragma unroll
+    for (int j = 0; j < kNM; ++j) red[j * 128 + nl] = __uint_as_float(r[j]);
+    // The warp's stores are ordered before lane 0's release arrivals (the
+    // warp barrier orders them; release is cumulative); each peer's acquiring
+    // wait then sees them.  A CTA that failed above still arrives, so its
+    // peers finish; the error word reports the call.
+    __syncwarp();
+    if (lane == 0)
+      for (int q = 0; q < ns; ++q) mbar_arrive_cluster(mapa_shared(smem_u32(red_ready), static_cast<uint32_t>(q)));
+    ok = mbar_wait_cluster(red_ready, 0, p.timeout_ns, abort_flag, kSiteClusterReduce) && ok;
+    if (ok) {
+      switch (ns) {
+        case 2: cluster_reduce_slice<2, kNM>(red, rank, first_tile, threadIdx.x - 64, p); break;
+        case 4: cluster_reduce_slice<4, kNM>(red, rank, first_tile, threadIdx.x - 64, p); break;
+        case 7: cluster_reduce_slice<7, kNM>(red, rank, first_tile, threadIdx.x - 64, p); break;
+        case 8: cluster_reduce_slice<8, kNM>(red, rank, first_tile, threadIdx.x - 64, p); break;
+        default: cluster_reduce_slice<3, kNM>(red, rank, first_tile, threadIdx.x - 64, p); break;  // 3, 5, 6
+      }
+    }
   } else if (warp < Cfg::kQuantWarp0) {
     // ------------------------------------------------------ epilogue
     griddep_wait();  // the workspace and C may still be in use by the preceding kernel
@@ -493,6 +622,7 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (kCR) cluster_sync_all();  // no CTA leaves while a peer may still read its partial
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::kTmemCols);

@@ -446,28 +446,51 @@ static size_t small_m_partials_bytes(int ctas, int nm) {
 // Launched with programmatic stream serialisation: the kernel may start while
 // the preceding kernel on the stream (normally the activation quantizer) is
 // still running; it prefetches weights and then waits for it in-kernel.
+// With p.cluster_s > 1 the kernel reduces split tiles inside clusters of
+// p.cluster_s CTAs (one cluster per weight tile) instead of the workspace.
 template <int kNM, bool kQX = false>
 static fp8mm_status launch_small_m_t(const CUtensorMap& tw, const CUtensorMap& tx, const DecodeArgs& p,
                                      cudaStream_t stream, int dev) {
   constexpr int kStages = kQX ? dec_stages_qx(kNM) : dec_stages(kNM);
   using Cfg = DecodeCfg<kNM, kStages, kQX>;
-  auto kern = gemm_small_m_kernel<kNM, kStages, kQX>;
+  const bool cr = p.cluster_s > 1;
+  auto kern = cr ? gemm_small_m_kernel<kNM, kStages, kQX, true> : gemm_small_m_kernel<kNM, kStages, kQX, false>;
   fp8mm_status st = ensure_smem(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, dev);
   if (st != FP8MM_OK) return st;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cr ? static_cast<unsigned>(p.cluster_s) : 1u;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.gridDim = dim3(p.ctas, 1, 1);
   cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cr ? 2 : 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tx, p);
   if (e != cudaSuccess) return cuda_fail(e);
   return launched();
 }
+
+// Largest cluster the small-M kernel reduces in (portable cluster size).
+constexpr int64_t kMaxClusterSplit = 8;
+
+// CTAs per weight tile when `ctas` is a tile-aligned split that the kernel can
+// reduce inside clusters (2..8 CTAs per tile, dividing the tile's K slabs);
+// 0 otherwise.
+static int cluster_split(int64_t ctas, int64_t n_tiles, int64_t num_k) {
+  if (ctas % n_tiles != 0) return 0;
+  const int64_t s = ctas / n_tiles;
+  return (s >= 2 && s <= kMaxClusterSplit && num_k % s == 0) ? static_cast<int>(s) : 0;
+}
+
+// Largest tile-aligned CTA count (s CTAs per tile, 2 <= s <= 8, s dividing
+// the K slabs, at least kMinSlabsPerCta slabs each) within `slots`; 0 if none.
+static int64_t best_cluster_ctas(int64_t n_tiles, int64_t num_k, int64_t slots);
 
 // Slabs per CTA (past the staged ones) whose weights the small-M kernel
 // prefetches into L2 when it starts.  Only where two CTAs share an SM: the
@@ -503,6 +526,12 @@ static int small_m_l2_ahead(int64_t units, int64_t ctas, int64_t sms) {
 // than both neighbours (e.g. 6144 x 4096, m = 1: 8.5 us at 192 CTAs, 9.6-10.4
 // us at 160-240).
 constexpr int64_t kMinSlabsPerCta = 4;
+static int64_t best_cluster_ctas(int64_t n_tiles, int64_t num_k, int64_t slots) {
+  int64_t best = 0;
+  for (int64_t s = 2; s <= kMaxClusterSplit && s <= num_k / kMinSlabsPerCta; ++s)
+    if (num_k % s == 0 && n_tiles * s <= slots) best = n_tiles * s;
+  return best;
+}
 static int small_m_ctas(int64_t units, int64_t n_tiles, int64_t num_k, int nm, int64_t requested, int64_t sms) {
   int64_t g = requested;
   if (g <= 0) {
@@ -538,15 +567,25 @@ static fp8mm_status launch_small_m(const void* a, const uint8_t* sfa, const void
   p.n_kc = p.num_k;
   p.timeout_ns = wait_timeout_ns();
   p.prefetch_w = (opt != nullptr && (opt->flags & FP8MM_FLAG_WEIGHTS_READY)) ? 1 : 0;
-  if (opt == nullptr || opt->workspace == nullptr) {
-    p.ctas = p.n_tiles;  // one CTA per weight tile, whole K: no partial sums
-  } else {
-    p.ctas = small_m_ctas(p.units, p.n_tiles, p.num_k, nm, opt->small_m_ctas, dev.sms);
-    const size_t need = fp8mm_workspace_bytes(m, n, k, p.ctas);
-    if (opt->workspace_bytes < need || !aligned(opt->workspace, 256)) return FP8MM_ERR_WORKSPACE;
-    p.partials = static_cast<float*>(opt->workspace);
-    p.tickets = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(opt->workspace) +
-                                            small_m_partials_bytes(p.ctas, nm));
+  const bool via_ws = opt != nullptr && (opt->flags & FP8MM_FLAG_SPLIT_VIA_WORKSPACE);
+  const int64_t requested = opt != nullptr ? opt->small_m_ctas : 0;
+  p.ctas = small_m_ctas(p.units, p.n_tiles, p.num_k, nm, requested, dev.sms);
+  p.cluster_s = via_ws ? 0 : cluster_split(p.ctas, p.n_tiles, p.num_k);
+  if (p.cluster_s == 0) {
+    if (opt != nullptr && opt->workspace != nullptr) {
+      const size_t need = fp8mm_workspace_bytes(m, n, k, p.ctas);
+      if (opt->workspace_bytes < need || !aligned(opt->workspace, 256)) return FP8MM_ERR_WORKSPACE;
+      p.partials = static_cast<float*>(opt->workspace);
+      p.tickets = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(opt->workspace) +
+                                              small_m_partials_bytes(p.ctas, nm));
+    } else {
+      // No workspace: a tile-aligned split reduced in clusters where one
+      // fits (automatic count only), else one CTA per weight tile over all
+      // of K (no partial sums).
+      const int64_t g = (requested > 0 || via_ws) ? 0 : best_cluster_ctas(p.n_tiles, p.num_k, dev.sms * (nm <= 32 ? 2 : 1));
+      p.ctas = static_cast<int>(g > 0 ? g : p.n_tiles);
+      p.cluster_s = g > 0 ? cluster_split(g, p.n_tiles, p.num_k) : 0;
+    }
   }
   p.l2_ahead = small_m_l2_ahead(p.units, p.ctas, dev.sms);
   CUtensorMap tw, tx;
@@ -972,6 +1011,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[FP8MM_NOALLOC_S
 // per device (host code may not use the symbol itself as a device pointer).
 static fp8mm_status noalloc_scratch(int dev, unsigned char** out) {
   static unsigned char* addr[64] = {};
+  if (dev < 0 || dev >= 64) return FP8MM_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
@@ -1017,11 +1057,14 @@ extern "C" fp8mm_status mxfp8_gemm_small_m_noalloc(const void* a_e4m3, const uin
   p.sfx = sf_a;
   p.n_kc = p.num_k;
   p.timeout_ns = wait_timeout_ns();
-  // as many CTAs as the partial-sum region holds (2 slots of 128 x nm fp32 each)
+  // mxfp8_gemm's automatic CTA count, capped at what the partial-sum region
+  // holds (2 slots of 128 x nm fp32 each)
   const int64_t per_cta = 2 * static_cast<int64_t>(nm) * 128 * static_cast<int64_t>(sizeof(float));
-  int64_t g = std::min<int64_t>(dev.sms, static_cast<int64_t>(kNoAllocPartialBytes) / per_cta);
+  int64_t g = small_m_ctas(p.units, p.n_tiles, p.num_k, nm, 0, dev.sms);
+  g = std::min<int64_t>(g, static_cast<int64_t>(kNoAllocPartialBytes) / per_cta);
   g = std::max<int64_t>(1, std::min<int64_t>(g, p.units));
   p.ctas = static_cast<int>(g);
+  p.cluster_s = cluster_split(g, p.n_tiles, p.num_k);  // tile-aligned: reduced in clusters, scratch unused
   p.partials = reinterpret_cast<float*>(scratch);
   p.tickets = reinterpret_cast<unsigned*>(scratch + kNoAllocPartialBytes);
   p.l2_ahead = small_m_l2_ahead(p.units, p.ctas, dev.sms);

@@ -21,6 +21,7 @@ enum DevErr : unsigned { kDevErrTimeout = 1 };
 enum WaitSite : unsigned {
   kSiteProducerEmpty = 1, kSiteMmaFull = 2, kSiteMmaAccEmpty = 3, kSiteEpiAccFull = 4,
   kSiteDrain = 5, kSiteProducerDrain = 6, kSiteSelfTest = 7, kSiteEpiSync = 8, kSiteQuantStage = 9,
+  kSiteClusterReduce = 10,
 };
 
 __device__ __forceinline__ void record_error(unsigned kind, unsigned site) {
@@ -224,6 +225,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t smem_addr, uint32_t ran
 }
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 32-bit load from the shared memory of a CTA of this cluster (an address
+// from mapa_shared).
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");

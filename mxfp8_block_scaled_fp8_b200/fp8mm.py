@@ -36,6 +36,7 @@ class Fp8mmError(RuntimeError):
 
 
 FLAG_WEIGHTS_READY = 1
+FLAG_SPLIT_VIA_WORKSPACE = 2
 
 
 class Opts(ctypes.Structure):
@@ -252,12 +253,14 @@ def quantize_gemm_workspace_bytes(m: int, n: int, k: int, ctas: int = 0) -> int:
 
 def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch.Tensor,
                c: torch.Tensor | None = None, workspace: torch.Tensor | None = None, kernel: int = KERNEL_AUTO,
-               small_m_ctas: int = 0, weights_ready: bool = False, stream=None) -> torch.Tensor:
+               small_m_ctas: int = 0, weights_ready: bool = False, stream=None,
+               split_via_workspace: bool = False) -> torch.Tensor:
     """C bf16 [m, n] = block-scaled A x B^T; a [m,k], b [n,k] codes with their library-layout scales.
     workspace (zeroed once, workspace_bytes(m, n, k, small_m_ctas) bytes): the small-M kernel's stream-K
-    split for m <= 64; for m > 64 the K split of shapes that fill less than one wave of SM pairs.
+    split for m <= 64 where the CTA count is not tile-aligned (aligned splits reduce inside clusters);
+    for m > 64 the K split of shapes that fill less than one wave of SM pairs.
     weights_ready: b and sf_b were complete before the preceding kernel on the stream started (see
-    FP8MM_FLAG_WEIGHTS_READY)."""
+    FP8MM_FLAG_WEIGHTS_READY).  split_via_workspace: FP8MM_FLAG_SPLIT_VIA_WORKSPACE."""
     a, b = _u8(a), _u8(b)
     _need(a, torch.uint8, "a"); _need(b, torch.uint8, "b")
     _need(sf_a, torch.uint8, "sf_a"); _need(sf_b, torch.uint8, "sf_b")
@@ -267,7 +270,8 @@ def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch
         raise ValueError("a [m,k] and b [n,k] must be contiguous with the same k")
     if c is None:
         c = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
-    opts = _ws_opts(workspace, kernel, small_m_ctas, FLAG_WEIGHTS_READY if weights_ready else 0)
+    flags = (FLAG_WEIGHTS_READY if weights_ready else 0) | (FLAG_SPLIT_VIA_WORKSPACE if split_via_workspace else 0)
+    opts = _ws_opts(workspace, kernel, small_m_ctas, flags)
     _check("mxfp8_gemm", lib().mxfp8_gemm(a.data_ptr(), sf_a.data_ptr(), b.data_ptr(), sf_b.data_ptr(), m, n, k,
                                           c.data_ptr(), _ld(c, "c"), ctypes.byref(opts), _stream(stream)))
     return c
@@ -275,7 +279,7 @@ def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch
 
 def mxfp8_quantize_gemm(a: torch.Tensor, b: torch.Tensor, sf_b: torch.Tensor, c: torch.Tensor | None = None,
                         workspace: torch.Tensor | None = None, kernel: int = KERNEL_AUTO, small_m_ctas: int = 0,
-                        weights_ready: bool = False, stream=None) -> torch.Tensor:
+                        weights_ready: bool = False, stream=None, split_via_workspace: bool = False) -> torch.Tensor:
     """C bf16 [m, n] = mxfp8_gemm(mxfp8_quantize(a), b) for m <= 64 from the bf16 activation a [m, k]:
     quantized inside the GEMM kernel for m <= 8, else by its own launch into the workspace tail
     (workspace of quantize_gemm_workspace_bytes(m, n, k, small_m_ctas) bytes, required for m > 8)."""
@@ -289,7 +293,8 @@ def mxfp8_quantize_gemm(a: torch.Tensor, b: torch.Tensor, sf_b: torch.Tensor, c:
         c = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
     opts = Opts(workspace.data_ptr() if workspace is not None else None,
                 workspace.numel() * workspace.element_size() if workspace is not None else 0,
-                kernel, small_m_ctas, FLAG_WEIGHTS_READY if weights_ready else 0)
+                kernel, small_m_ctas,
+                (FLAG_WEIGHTS_READY if weights_ready else 0) | (FLAG_SPLIT_VIA_WORKSPACE if split_via_workspace else 0))
     _check("mxfp8_quantize_gemm", lib().mxfp8_quantize_gemm(
         a.data_ptr(), _ld(a, "a"), b.data_ptr(), sf_b.data_ptr(), m, n, k, c.data_ptr(), _ld(c, "c"),
         ctypes.byref(opts), _stream(stream)))

@@ -145,5 +145,64 @@ def test_workspace_too_small_is_rejected(decode_data):
     n, k = synthetic.DECODE_SHAPES["qkv"]
     gx, gsfx = fp8mm.mxfp8_quantize(gu.to_dev(xs[k][:8].contiguous()))
     ws = torch.zeros(1024, dtype=torch.uint8, device="cuda")
-    with pytest.raises(fp8mm.Fp8mmError):
-        fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws)
+    with pytest.raises(fp8mm.Fp8mmError):                       # a split reduced through the workspace
+        fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, split_via_workspace=True)
+    with pytest.raises(fp8mm.Fp8mmError):                       # 37 CTAs: not tile-aligned
+        fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, small_m_ctas=37)
+
+
+# ------------------------------------------------------------ tile-aligned splits reduced in clusters
+
+N_TILES = {name: -(-n // 128) for name, (n, k) in synthetic.DECODE_SHAPES.items()}
+
+
+@pytest.mark.parametrize("name,m,s", [("qkv", 1, 4), ("qkv", 64, 2), ("up", 8, 2), ("up", 32, 4), ("up", 64, 8),
+                                      ("down", 1, 8), ("down", 16, 7), ("down", 48, 4), ("down", 64, 2)])
+def test_cluster_reduction_equals_workspace_reduction(decode_data, name, m, s):
+    """s CTAs per weight tile (2 <= s <= 8, s dividing the tile's K slabs:
+    32 for up and qkv, 112 for down) are reduced inside a cluster through
+    distributed shared memory; the same partition reduced through the
+    workspace gives identical bits, and both meet the bar."""
+    import oracle as orc
+    weights, xs = decode_data
+    qw, sfw, gw, gsfw = weights[name]
+    n, k = synthetic.DECODE_SHAPES[name]
+    ctas = N_TILES[name] * s
+    x = xs[k][:m].contiguous()
+    qx, sfx = orc.mx_quantize(synthetic.bits(x))
+    gx, gsfx = fp8mm.mxfp8_quantize(gu.to_dev(x))
+    ws = _workspace(m, n, k, ctas)
+    c_cl = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, small_m_ctas=ctas, weights_ready=True)   # no workspace needed
+    c_cl2 = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, small_m_ctas=ctas)
+    torch.cuda.synchronize()
+    assert not ws.any()                                          # the cluster path leaves a workspace alone
+    c_ws = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, small_m_ctas=ctas, split_via_workspace=True)
+    torch.cuda.synchronize()
+    c_ref, bound = orc.gemm_mx(qx, sfx, qw, sfw)
+    gu.check_gemm(c_cl, c_ref, bound, f"cluster reduction {name} m={m} s={s}")
+    assert torch.equal(c_cl, c_ws) and torch.equal(c_cl, c_cl2)
+    tickets = -(-N_TILES[name] * 4 // 256) * 256
+    assert not ws[-tickets:].any()                               # the workspace path reset its counters
+    assert fp8mm.last_device_error() == 0
+
+
+@pytest.mark.parametrize("m,n,k,s", [(5, 200, 512, 2), (17, 130, 4096, 8), (40, 384, 896, 7), (64, 257, 1024, 4)])
+def test_cluster_reduction_ragged(m, n, k, s):
+    """Ragged weight tiles (n not a multiple of 128) and token counts that fill
+    part of the 16/32/48/64-token tile, with 2, 4, 7 and 8 CTAs per tile."""
+    import oracle as orc
+    x = synthetic.random_bf16((m, k), seed=m * 7 + k)
+    w = synthetic.random_bf16((n, k), seed=n * 11 + k, sigma=0.02)
+    qx, sfx = orc.mx_quantize(synthetic.bits(x))
+    qw, sfw = orc.mx_quantize(synthetic.bits(w))
+    gx, gsfx = fp8mm.mxfp8_quantize(gu.to_dev(x))
+    gw, gsfw = fp8mm.mxfp8_quantize(gu.to_dev(w))
+    ctas = -(-n // 128) * s
+    c = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, small_m_ctas=ctas)
+    ws = _workspace(m, n, k, ctas)
+    c_ws = fp8mm.mxfp8_gemm(gx, gsfx, gw, gsfw, workspace=ws, small_m_ctas=ctas, split_via_workspace=True)
+    torch.cuda.synchronize()
+    c_ref, bound = orc.gemm_mx(qx, sfx, qw, sfw)
+    gu.check_gemm(c, c_ref, bound, f"cluster reduction ragged {m}x{n}x{k} s={s}")
+    assert torch.equal(c, c_ws)
+    assert fp8mm.last_device_error() == 0

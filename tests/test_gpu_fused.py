@@ -170,8 +170,11 @@ def test_fused_degenerate_and_errors(weights):
     x = gu.to_dev(synthetic.random_bf16((65, k), seed=65))
     with pytest.raises(fp8mm.Fp8mmError):
         fp8mm.mxfp8_quantize_gemm(x, gw, gsfw)                  # m > 64
-    with pytest.raises(fp8mm.Fp8mmError):
-        fp8mm.mxfp8_quantize_gemm(x[:8], gw, gsfw, workspace=torch.zeros(256, dtype=torch.uint8, device="cuda"))
+    tiny_ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fp8mm.Fp8mmError):                          # a split reduced through the workspace
+        fp8mm.mxfp8_quantize_gemm(x[:8], gw, gsfw, workspace=tiny_ws, split_via_workspace=True)
+    with pytest.raises(fp8mm.Fp8mmError):                          # 37 CTAs: not tile-aligned
+        fp8mm.mxfp8_quantize_gemm(x[:8], gw, gsfw, workspace=tiny_ws, small_m_ctas=37)
     with pytest.raises(fp8mm.Fp8mmError):
         fp8mm.mxfp8_quantize_gemm(x[:8], gw, gsfw, kernel=fp8mm.KERNEL_TILED)
     with pytest.raises(fp8mm.Fp8mmError):                          # m > 8 without room for the activation
