@@ -113,6 +113,10 @@ typedef struct fp8mm_opts {
  * then needs no workspace.  With this flag it reduces such splits through
  * the workspace instead (identical results; for comparison and testing). */
 #define FP8MM_FLAG_SPLIT_VIA_WORKSPACE 2u
+/* mxfp8_gemm / small-M kernel only (m <= 64; FP8MM_ERR_SHAPE otherwise):
+ * sf_a is in the small-M scale layout written by mxfp8_quantize_8x4 instead
+ * of the 128-row chunk layout. */
+#define FP8MM_FLAG_SF_A_8X4 4u
 
 #define FP8MM_KERNEL_AUTO 0
 #define FP8MM_KERNEL_TILED 1
@@ -217,6 +221,24 @@ fp8mm_status fp8mm_sf_from_canonical(const uint8_t* canonical, int64_t rows, int
  * q 8-byte aligned, sf 16-byte aligned.  rows == 0 or k == 0 is a no-op. */
 fp8mm_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, void* q_e4m3,
                             int64_t ld_q, uint8_t* sf, void* stream);
+
+/* Small-M scale layout, for activations of a few token rows -- the
+ * use_8x4_sf_layout option of the mm_mxfp8 call on page "[sglang] FlashInfer
+ * v0.6.7 MXFP8 Gemm 통합", section 2, in this library's own form: rows are
+ * padded to a multiple of 8 (not 128) and K-blocks to a multiple of 4.  The
+ * buffer is made of 32-byte atoms of 8 rows x 4 K-blocks; atom (r8, g) sits at
+ * (g * ceil(rows / 8) + r8) * 32, and inside it the byte of row r and block b
+ * is (r % 8) * 4 + (b % 4).  So for each 128-wide K slab g the 32-bit scale
+ * words of all rows are contiguous: byte ((b / 4) * rows_pad8 + r) * 4 + b % 4.
+ * Padding bytes are written as 0.  Byte value e encodes 2^(e - 127). */
+size_t fp8mm_sf8x4_bytes(int64_t rows, int64_t k);
+/* Byte offset of (row, block) in the small-M layout; -1 when out of range. */
+int64_t fp8mm_sf8x4_offset(int64_t rows, int64_t k, int64_t row, int64_t block);
+/* mxfp8_quantize with the scales in the small-M layout (sf:
+ * fp8mm_sf8x4_bytes(rows, k) bytes, written whole, padding included); the
+ * codes and exponents are those of mxfp8_quantize.  Same arguments and rules. */
+fp8mm_status mxfp8_quantize_8x4(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, void* q_e4m3,
+                                int64_t ld_q, uint8_t* sf, void* stream);
 
 /* MXFP8 block-scaled GEMM (mode 2) -- the mm_mxfp8(a, b_t, a_sf, b_sf,
  * out_dtype=bf16) call of page "[sglang] FlashInfer v0.6.7 MXFP8 Gemm 통합",

@@ -25,6 +25,14 @@
 // workspace and no global round trip; the cluster meets once more before
 // exit so that no CTA leaves while a peer may still read its shared memory.
 //
+// With kSF8 the activation's scales come in the small-M ("8x4") layout of
+// mxfp8_quantize_8x4: per 128-wide K slab one 32-bit word per token row
+// (rows padded to 8), rows_pad8 * 4 contiguous bytes, instead of the 512-byte
+// chunk of 128 rows.  One more warp reads each slab's words (L2-resident) and
+// writes them into the stage's scale image in the chunk form tcgen05.cp
+// takes (row r at byte (r % 32) * 16 + (r / 32) * 4), then arrives on the
+// stage's full barrier next to the TMA bytes.
+//
 // With kQX (m <= 8) the activation arrives as bf16 and is quantized inside
 // the kernel (the per-call activation quantization of page "[sglang]
 // FlashInfer v0.6.7 MXFP8 Gemm 통합", section 2, fused into the GEMM): two
@@ -72,11 +80,13 @@ struct DecodeArgs {
   int cluster_s;           // kCR: CTAs per weight tile (= the cluster size)
 };
 
-template <int kNM, int kStages, bool kQX = false>
+template <int kNM, int kStages, bool kQX = false, bool kSF8 = false>
 struct DecodeCfg {
   static_assert(kNM % 16 == 0 && kNM >= 16 && kNM <= 64, "token tile");
-  // warps: producer, MMA, four epilogue warps (+ two activation-quantizer warps)
-  static constexpr int kQuantWarps = kQX ? 2 : 0;
+  static_assert(!(kQX && kSF8), "the in-kernel quantizer writes the scale image itself");
+  // warps: producer, MMA, four epilogue warps (+ two activation-quantizer
+  // warps, or one warp that lays out 8x4 activation scales)
+  static constexpr int kQuantWarps = kQX ? 2 : (kSF8 ? 1 : 0);
   static constexpr int kThreads = 192 + 32 * kQuantWarps;
   static constexpr int kQuantWarp0 = 6;
   // Token tiles up to 32 keep shared memory and registers within half an SM,
@@ -195,12 +205,12 @@ __device__ __forceinline__ void cluster_reduce_slice(const float* red, int rank,
 
 // tmX: the quantized activation (E4M3 [m, k], 128-byte swizzle, box 128 x
 // kNM); unused with kQX (the activation comes as p.x).
-template <int kNM, int kStages, bool kQX, bool kCR = false>
-__global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
-                                  DecodeCfg<kNM, kStages, kQX>::kMinBlocksPerSm)
+template <int kNM, int kStages, bool kQX, bool kCR = false, bool kSF8 = false>
+__global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX, kSF8>::kThreads,
+                                  DecodeCfg<kNM, kStages, kQX, kSF8>::kMinBlocksPerSm)
     gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                         const DecodeArgs p) {
-  using Cfg = DecodeCfg<kNM, kStages, kQX>;
+  using Cfg = DecodeCfg<kNM, kStages, kQX, kSF8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
@@ -224,7 +234,7 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], kQX ? 2 : 1);  // kQX: the weight bytes and the quantizer warp
+      mbar_init(&full[s], (kQX || kSF8) ? 2 : 1);  // + the quantizer (kQX) or scale (kSF8) warp
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -265,7 +275,9 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
       const int npre = static_cast<int>(nslabs < kStages ? nslabs : kStages);
       const int t0 = static_cast<int>(u_begin / p.num_k);
       const int kb0 = static_cast<int>(u_begin % p.num_k);
-      constexpr uint32_t kTx = kQX ? Cfg::kWBytes + 512u : Cfg::kWBytes + Cfg::kXBytes + 1024u;
+      constexpr uint32_t kTx = kQX    ? Cfg::kWBytes + 512u
+                               : kSF8 ? Cfg::kWBytes + Cfg::kXBytes + 512u
+                                      : Cfg::kWBytes + Cfg::kXBytes + 1024u;
       int t = t0, kb = kb0;
       for (int i = 0; i < npre; ++i) {  // fresh stages: nothing to wait for
         mbar_arrive_expect_tx(&full[i], kTx);
@@ -294,7 +306,8 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
       for (int i = 0; i < npre; ++i) {
         if (!kQX) {
           tma_load_2d(smem + Cfg::kOffX + i * Cfg::kXBytes, &tmX, &full[i], kb * 128, 0);
-          bulk_load(smem + Cfg::kOffSfx + i * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[i]);
+          if (!kSF8)
+            bulk_load(smem + Cfg::kOffSfx + i * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[i]);
         }
         if (++kb == p.num_k) {
           kb = 0;
@@ -313,7 +326,9 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
                   &full[stage]);
         if (!kQX) {
           tma_load_2d(smem + Cfg::kOffX + stage * Cfg::kXBytes, &tmX, &full[stage], kb * 128, 0);
-          bulk_load(smem + Cfg::kOffSfx + stage * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[stage]);
+          if (!kSF8)
+            bulk_load(smem + Cfg::kOffSfx + stage * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u,
+                      &full[stage]);
         }
         issued_mask |= 1u << stage;
         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -617,6 +632,49 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX>::kThreads,
           cur[q][t] = nxt[q][t];
           nxt[q][t] = nxt2[q][t];
         }
+    }
+  }
+
+  if constexpr (kSF8) {
+    if (warp == Cfg::kQuantWarp0) {
+      // ---------------------------------------------------- 8x4 activation scales
+      // Lane L owns token rows L and L + 32: its word of each slab goes to
+      // the image at byte L * 16 (row L) and L * 16 + 4 (row L + 32).  Words
+      // of rows past m are zero in the 8x4 layout up to rows_pad8, and zero
+      // here beyond it; rows >= kNM are never read.  The next two slabs'
+      // words are in flight while the current one is placed.
+      constexpr int kW = kNM > 32 ? 2 : 1;
+      const int rows8 = (p.m + 7) & ~7;
+      const int64_t nslabs = u_end - u_begin;
+      griddep_wait();  // the scales may be written by the preceding kernel
+      auto load = [&](int64_t i, uint32_t (&w)[kW]) {
+        const int kb = static_cast<int>((u_begin + i) % p.num_k);
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(p.sfx) + static_cast<int64_t>(kb) * rows8;
+#pragma unroll
+        for (int h = 0; h < kW; ++h) w[h] = (lane + 32 * h < rows8) ? __ldcg(src + lane + 32 * h) : 0u;
+      };
+      uint32_t cur[kW], nxt[kW], nxt2[kW];
+      if (nslabs > 0) load(0, cur);
+      if (nslabs > 1) load(1, nxt);
+      bool ok = true;
+      for (int64_t i = 0; i < nslabs; ++i) {
+        if (i + 2 < nslabs) load(i + 2, nxt2);
+        const int stage = static_cast<int>(i % kStages);
+        ok = ok && mbar_wait(&empty[stage], static_cast<uint32_t>(((i / kStages) & 1) ^ 1), p.timeout_ns,
+                             abort_flag, kSiteQuantStage);
+        if (!__all_sync(0xFFFFFFFFu, ok)) break;
+        uint32_t* img = reinterpret_cast<uint32_t*>(smem + Cfg::kOffSfx + stage * 512);
+#pragma unroll
+        for (int h = 0; h < kW; ++h) img[lane * 4 + h] = cur[h];
+        fence_proxy_async_smem();  // the image is read by tcgen05.cp (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);
+#pragma unroll
+        for (int h = 0; h < kW; ++h) {
+          cur[h] = nxt[h];
+          nxt[h] = nxt2[h];
+        }
+      }
     }
   }
 

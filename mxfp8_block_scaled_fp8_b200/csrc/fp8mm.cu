@@ -448,13 +448,15 @@ static size_t small_m_partials_bytes(int ctas, int nm) {
 // still running; it prefetches weights and then waits for it in-kernel.
 // With p.cluster_s > 1 the kernel reduces split tiles inside clusters of
 // p.cluster_s CTAs (one cluster per weight tile) instead of the workspace.
-template <int kNM, bool kQX = false>
+// kSF8: the activation's scales are in the small-M (8x4) layout.
+template <int kNM, bool kQX = false, bool kSF8 = false>
 static fp8mm_status launch_small_m_t(const CUtensorMap& tw, const CUtensorMap& tx, const DecodeArgs& p,
                                      cudaStream_t stream, int dev) {
   constexpr int kStages = kQX ? dec_stages_qx(kNM) : dec_stages(kNM);
-  using Cfg = DecodeCfg<kNM, kStages, kQX>;
+  using Cfg = DecodeCfg<kNM, kStages, kQX, kSF8>;
   const bool cr = p.cluster_s > 1;
-  auto kern = cr ? gemm_small_m_kernel<kNM, kStages, kQX, true> : gemm_small_m_kernel<kNM, kStages, kQX, false>;
+  auto kern = cr ? gemm_small_m_kernel<kNM, kStages, kQX, true, kSF8>
+                 : gemm_small_m_kernel<kNM, kStages, kQX, false, kSF8>;
   fp8mm_status st = ensure_smem(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, dev);
   if (st != FP8MM_OK) return st;
   cudaLaunchConfig_t cfg = {};
@@ -597,6 +599,14 @@ static fp8mm_status launch_small_m(const void* a, const uint8_t* sfa, const void
     p.ldx = lda;
     return launch_small_m_t<16, true>(tw, tw, p, stream, dev.device);
   }
+  if (opt != nullptr && (opt->flags & FP8MM_FLAG_SF_A_8X4)) {
+    switch (nm) {
+      case 16: return launch_small_m_t<16, false, true>(tw, tx, p, stream, dev.device);
+      case 32: return launch_small_m_t<32, false, true>(tw, tx, p, stream, dev.device);
+      case 48: return launch_small_m_t<48, false, true>(tw, tx, p, stream, dev.device);
+      default: return launch_small_m_t<64, false, true>(tw, tx, p, stream, dev.device);
+    }
+  }
   switch (nm) {
     case 16: return launch_small_m_t<16>(tw, tx, p, stream, dev.device);
     case 32: return launch_small_m_t<32>(tw, tx, p, stream, dev.device);
@@ -727,8 +737,12 @@ fp8mm_status fp8_tensor_scale(const void* x_bf16, int64_t rows, int64_t k, int64
   cudaError_t e = cudaMemsetAsync(scale, 0, sizeof(float), s);
   if (e != cudaSuccess) return cuda_fail(e);
   if (rows > 0 && k > 0) {
-    const int64_t vecs = rows * (k / 8);
-    const int grid = static_cast<int>(std::min<int64_t>(cdiv(vecs, kTensorThreads), static_cast<int64_t>(dev.sms) * 8));
+    // contiguous tensors are one flat run of vectors, strided ones go row by
+    // row; at most eight blocks per SM
+    const int64_t per_block = kTensorThreads * kAmaxUnroll;
+    const int64_t want = ld_x == k ? cdiv(rows * (k / 8), per_block)
+                                   : cdiv(rows, std::max<int64_t>(1, cdiv(per_block, k / 8)));
+    const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(dev.sms) * 8));
     st = launch_pdl(tensor_amax_kernel, dim3(grid), dim3(kTensorThreads), 0, s,
                     static_cast<const __nv_bfloat16*>(x_bf16), rows, k, ld_x, reinterpret_cast<unsigned*>(scale));
     if (st != FP8MM_OK) return st;
@@ -770,7 +784,39 @@ fp8mm_status mxfp8_quantize(const void* x_bf16, int64_t rows, int64_t k, int64_t
   // one warp per 32-block segment of a padded row, 8 warps per CTA
   const int64_t segments = rows_pad * cdiv(cdiv(k, 128) * 4, 32);
   const int grid = static_cast<int>(std::min<int64_t>(cdiv(segments, kQ2Threads / 32), static_cast<int64_t>(dev.sms) * 8));
-  st = launch_pdl(quant_mx_kernel, dim3(grid), dim3(kQ2Threads), 0, static_cast<cudaStream_t>(stream),
+  st = launch_pdl(quant_mx_kernel<false>, dim3(grid), dim3(kQ2Threads), 0, static_cast<cudaStream_t>(stream),
+                  static_cast<const __nv_bfloat16*>(x_bf16), rows, k, ld_x, static_cast<uint8_t*>(q_e4m3), ld_q, sf,
+                  static_cast<int>(n_kc), rows_pad);
+  return st != FP8MM_OK ? st : launched();
+}
+
+size_t fp8mm_sf8x4_bytes(int64_t rows, int64_t k) {
+  if (rows <= 0 || k <= 0) return 0;
+  return static_cast<size_t>(cdiv(rows, 8) * 8) * static_cast<size_t>(cdiv(k, 128)) * 4;
+}
+
+int64_t fp8mm_sf8x4_offset(int64_t rows, int64_t k, int64_t row, int64_t block) {
+  if (rows <= 0 || k <= 0) return -1;
+  const int64_t rows8 = cdiv(rows, 8) * 8;
+  if (row < 0 || row >= rows8 || block < 0 || block >= cdiv(k, 128) * 4) return -1;
+  return ((block / 4) * rows8 + row) * 4 + block % 4;
+}
+
+fp8mm_status mxfp8_quantize_8x4(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, void* q_e4m3,
+                                int64_t ld_q, uint8_t* sf, void* stream) {
+  if (rows < 0 || k < 0 || k % 32 != 0 || ld_x < k || ld_q < k) return FP8MM_ERR_SHAPE;
+  if (rows == 0 || k == 0) return FP8MM_OK;
+  if (x_bf16 == nullptr || q_e4m3 == nullptr || sf == nullptr) return FP8MM_ERR_NULL;
+  if (!aligned(x_bf16, 16) || !aligned(q_e4m3, 8) || !aligned(sf, 16) || ld_x % 8 != 0 || ld_q % 8 != 0)
+    return FP8MM_ERR_ALIGN;
+  DeviceInfo dev;
+  fp8mm_status st = current_device(&dev);
+  if (st != FP8MM_OK) return st;
+  const int64_t n_kc = cdiv(k, 128);
+  const int64_t rows_pad = cdiv(rows, 8) * 8;
+  const int64_t segments = rows_pad * cdiv(n_kc * 4, 32);
+  const int grid = static_cast<int>(std::min<int64_t>(cdiv(segments, kQ2Threads / 32), static_cast<int64_t>(dev.sms) * 8));
+  st = launch_pdl(quant_mx_kernel<true>, dim3(grid), dim3(kQ2Threads), 0, static_cast<cudaStream_t>(stream),
                   static_cast<const __nv_bfloat16*>(x_bf16), rows, k, ld_x, static_cast<uint8_t*>(q_e4m3), ld_q, sf,
                   static_cast<int>(n_kc), rows_pad);
   return st != FP8MM_OK ? st : launched();
@@ -860,6 +906,10 @@ fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e
   const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
   if (kind == FP8MM_KERNEL_SMALL_M && m > 64) return FP8MM_ERR_SHAPE;
   if (kind < FP8MM_KERNEL_AUTO || kind > FP8MM_KERNEL_TILED_1SM_N128) return FP8MM_ERR_SHAPE;
+  // the 8x4 activation-scale layout is read by the small-M kernel only
+  if (opt != nullptr && (opt->flags & FP8MM_FLAG_SF_A_8X4) &&
+      !(kind == FP8MM_KERNEL_SMALL_M || (kind == FP8MM_KERNEL_AUTO && m <= 64)))
+    return FP8MM_ERR_SHAPE;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != FP8MM_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

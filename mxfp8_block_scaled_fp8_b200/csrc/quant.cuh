@@ -210,26 +210,57 @@ __global__ void __launch_bounds__(kQ1Threads) quant_rowwise_2pass_kernel(const _
 // ------------------------------------------------------------------ per tensor
 
 // Per-tensor scale (page "FP8 推理基础设施（五）：从 DeepGEMM 到 vLLM", listing 3:
-// one scale per tensor, max|x| / 448), in two steps: every warp takes the
-// exact maximum of |x| over its vectors (an unsigned 16-bit max over the
-// sign-cleared bf16 bits) and folds it into *word with atomicMax (the word
-// was zeroed; bf16 bits << 16 are the fp32 bits of the maximum, whose integer
-// order is their value order); then one thread turns it into
-// s = amax / 448 (IEEE division), 1 for an all-zero tensor.
+// one scale per tensor, max|x| / 448), in two kernels after a zeroing memset
+// of the output word: every block takes the exact maximum of |x| over its
+// share (an unsigned 16-bit max over the sign-cleared bf16 bits, four 16-byte
+// loads in flight per thread: one flat run for a contiguous tensor, row by
+// row otherwise) and folds it into the word with one atomicMax (bf16 bits
+// << 16 are the fp32 bits of the maximum, whose integer order is their value
+// order); then one thread turns it into s = amax / 448 (IEEE division), 1 for
+// an all-zero tensor.  A single-kernel form that finalized in the last block
+// to arrive (a compare-and-swap loop on the same word carrying an arrival
+// count in its low half) measured 16 times slower on B200: the blocks finish
+// together and their compare-and-swaps serialise.
 constexpr int kTensorThreads = 256;
+constexpr int kAmaxUnroll = 4;
 
 __global__ void __launch_bounds__(kTensorThreads) tensor_amax_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
                                                                     int64_t k, int64_t ld_x, unsigned* word) {
   griddep_launch_dependents();
   griddep_wait();
-  const uint32_t vpr = static_cast<uint32_t>(k / 8);  // 16-byte vectors per row
-  const uint32_t total = static_cast<uint32_t>(rows) * vpr;  // < 2^32 (checked by the host)
+  const int vpr = static_cast<int>(k / 8);  // 16-byte vectors per row
   uint32_t m = 0;
-  for (uint32_t v = blockIdx.x * kTensorThreads + threadIdx.x; v < total; v += gridDim.x * kTensorThreads) {
-    const uint32_t r = v / vpr;
-    const uint4 w = ld_stream_16(x + static_cast<int64_t>(r) * ld_x + (v - r * vpr) * 8);
-    m = __vmaxu2(__vmaxu2(m, w.x & 0x7FFF7FFFu),
-                 __vmaxu2(w.y & 0x7FFF7FFFu, __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
+  auto fold = [&m](const uint4& w) {
+    m = __vmaxu2(__vmaxu2(m, w.x & 0x7FFF7FFFu), __vmaxu2(w.y & 0x7FFF7FFFu, __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));
+  };
+  if (ld_x == k) {  // contiguous: one flat run of rows * k / 8 vectors
+    const int64_t total = rows * vpr;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kTensorThreads * kAmaxUnroll;
+    for (int64_t v0 = static_cast<int64_t>(blockIdx.x) * kTensorThreads * kAmaxUnroll + threadIdx.x; v0 < total;
+         v0 += stride) {
+      uint4 w[kAmaxUnroll];
+#pragma unroll
+      for (int u = 0; u < kAmaxUnroll; ++u) {
+        const int64_t v = v0 + u * kTensorThreads;
+        w[u] = v < total ? ld_stream_16(x + v * 8) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kAmaxUnroll; ++u) fold(w[u]);
+    }
+  } else {
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const __nv_bfloat16* xr = x + row * ld_x;
+    for (int v0 = threadIdx.x; v0 < vpr; v0 += kTensorThreads * kAmaxUnroll) {
+      uint4 w[kAmaxUnroll];
+#pragma unroll
+      for (int u = 0; u < kAmaxUnroll; ++u) {
+        const int v = v0 + u * kTensorThreads;
+        w[u] = v < vpr ? ld_stream_16(xr + static_cast<int64_t>(v) * 8) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kAmaxUnroll; ++u) fold(w[u]);
+    }
+  }
   }
   m = max(m & 0xFFFFu, m >> 16) << 16;
   m = __reduce_max_sync(0xFFFFFFFFu, m);
@@ -309,7 +340,10 @@ __device__ __forceinline__ float bf16x32_absmax(const uint4 (&v)[4]) {
 // exponent, 32 E4M3 bytes, and the lanes L % 4 == 0 gather the four
 // exponents of one scale word.  The next segment's loads are in flight
 // while the current one is converted.  Rows >= rows and blocks >= k/32
-// (padding) get exponent 0 and no codes.
+// (padding) get exponent 0 and no codes.  k8x4: the scales go to the small-M
+// layout (rows padded to 8; the word of row r and K group g at
+// (g * rows_pad + r) * 4) instead of the 128-row chunks.
+template <bool k8x4 = false>
 __global__ void __launch_bounds__(kQ2Threads) quant_mx_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
                                                               int64_t k, int64_t ld_x, uint8_t* __restrict__ q,
                                                               int64_t ld_q, uint8_t* __restrict__ sf, int n_kc,
@@ -373,9 +407,11 @@ __global__ void __launch_bounds__(kQ2Threads) quant_mx_kernel(const __nv_bfloat1
     const uint32_t e1 = __shfl_down_sync(0xFFFFFFFFu, static_cast<uint32_t>(e), 1);
     const uint32_t e2 = __shfl_down_sync(0xFFFFFFFFu, static_cast<uint32_t>(e), 2);
     const uint32_t e3 = __shfl_down_sync(0xFFFFFFFFu, static_cast<uint32_t>(e), 3);
-    if ((lane & 3) == 0 && kb < nkb4)
-      *reinterpret_cast<uint32_t*>(sf + ((row / 128) * n_kc + kb / 4) * 512 + (row % 32) * 16 + ((row % 128) / 32) * 4) =
-          static_cast<uint32_t>(e) | (e1 << 8) | (e2 << 16) | (e3 << 24);
+    if ((lane & 3) == 0 && kb < nkb4) {
+      const int64_t off = k8x4 ? (static_cast<int64_t>(kb / 4) * rows_pad + row) * 4
+                               : ((row / 128) * n_kc + kb / 4) * 512 + (row % 32) * 16 + ((row % 128) / 32) * 4;
+      *reinterpret_cast<uint32_t*>(sf + off) = static_cast<uint32_t>(e) | (e1 << 8) | (e2 << 16) | (e3 << 24);
+    }
 #pragma unroll
     for (int t = 0; t < 4; ++t) cur[t] = nxt[t];
     row = nrow;

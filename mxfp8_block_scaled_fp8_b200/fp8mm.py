@@ -37,6 +37,7 @@ class Fp8mmError(RuntimeError):
 
 FLAG_WEIGHTS_READY = 1
 FLAG_SPLIT_VIA_WORKSPACE = 2
+FLAG_SF_A_8X4 = 4
 
 
 class Opts(ctypes.Structure):
@@ -59,6 +60,9 @@ _SIGNATURES = {
     "concat_mla_k": ([_P, _P, _P] + [_I64] * 11 + [_P], ctypes.c_int),
     "fp8mm_sf_bytes": ([_I64, _I64], ctypes.c_size_t),
     "fp8mm_sf_offset": ([_I64, _I64, _I64, _I64], ctypes.c_int64),
+    "fp8mm_sf8x4_bytes": ([_I64, _I64], ctypes.c_size_t),
+    "fp8mm_sf8x4_offset": ([_I64, _I64, _I64, _I64], ctypes.c_int64),
+    "mxfp8_quantize_8x4": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P], ctypes.c_int),
     "fp8mm_sf_to_canonical": ([_P, _I64, _I64, _P], ctypes.c_int),
     "fp8mm_sf_from_canonical": ([_P, _I64, _I64, _P], ctypes.c_int),
     "fp8mm_workspace_bytes": ([_I64, _I64, _I64, ctypes.c_int32], ctypes.c_size_t),
@@ -243,6 +247,30 @@ def mxfp8_quantize(x: torch.Tensor, q: torch.Tensor | None = None, sf: torch.Ten
     return q, sf
 
 
+def sf8x4_bytes(rows: int, k: int) -> int:
+    return int(lib().fp8mm_sf8x4_bytes(rows, k))
+
+
+def sf8x4_offset(rows: int, k: int, row: int, block: int) -> int:
+    return int(lib().fp8mm_sf8x4_offset(rows, k, row, block))
+
+
+def mxfp8_quantize_8x4(x: torch.Tensor, q: torch.Tensor | None = None, sf: torch.Tensor | None = None,
+                       stream=None):
+    """mxfp8_quantize with the scales in the small-M (8x4) layout: (codes uint8 [rows, k],
+    scales uint8 [sf8x4_bytes]); for activations of a few token rows fed to mxfp8_gemm(sf_a_8x4=True)."""
+    _need(x, torch.bfloat16, "x")
+    rows, k = x.shape
+    if q is None:
+        q = torch.empty((rows, k), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty((max(sf8x4_bytes(rows, k), 1),), dtype=torch.uint8, device=x.device)
+    q = _u8(q)
+    _check("mxfp8_quantize_8x4", lib().mxfp8_quantize_8x4(x.data_ptr(), rows, k, _ld(x, "x"), q.data_ptr(),
+                                                          _ld(q, "q"), sf.data_ptr(), _stream(stream)))
+    return q, sf
+
+
 def workspace_bytes(m: int, n: int, k: int, ctas: int = 0) -> int:
     return int(lib().fp8mm_workspace_bytes(m, n, k, ctas))
 
@@ -254,13 +282,14 @@ def quantize_gemm_workspace_bytes(m: int, n: int, k: int, ctas: int = 0) -> int:
 def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch.Tensor,
                c: torch.Tensor | None = None, workspace: torch.Tensor | None = None, kernel: int = KERNEL_AUTO,
                small_m_ctas: int = 0, weights_ready: bool = False, stream=None,
-               split_via_workspace: bool = False) -> torch.Tensor:
+               split_via_workspace: bool = False, sf_a_8x4: bool = False) -> torch.Tensor:
     """C bf16 [m, n] = block-scaled A x B^T; a [m,k], b [n,k] codes with their library-layout scales.
     workspace (zeroed once, workspace_bytes(m, n, k, small_m_ctas) bytes): the small-M kernel's stream-K
     split for m <= 64 where the CTA count is not tile-aligned (aligned splits reduce inside clusters);
     for m > 64 the K split of shapes that fill less than one wave of SM pairs.
     weights_ready: b and sf_b were complete before the preceding kernel on the stream started (see
-    FP8MM_FLAG_WEIGHTS_READY).  split_via_workspace: FP8MM_FLAG_SPLIT_VIA_WORKSPACE."""
+    FP8MM_FLAG_WEIGHTS_READY).  split_via_workspace: FP8MM_FLAG_SPLIT_VIA_WORKSPACE.  sf_a_8x4: sf_a is in
+    the small-M layout of mxfp8_quantize_8x4 (m <= 64 only)."""
     a, b = _u8(a), _u8(b)
     _need(a, torch.uint8, "a"); _need(b, torch.uint8, "b")
     _need(sf_a, torch.uint8, "sf_a"); _need(sf_b, torch.uint8, "sf_b")
@@ -270,7 +299,8 @@ def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch
         raise ValueError("a [m,k] and b [n,k] must be contiguous with the same k")
     if c is None:
         c = torch.empty((m, n), dtype=torch.bfloat16, device=a.device)
-    flags = (FLAG_WEIGHTS_READY if weights_ready else 0) | (FLAG_SPLIT_VIA_WORKSPACE if split_via_workspace else 0)
+    flags = ((FLAG_WEIGHTS_READY if weights_ready else 0) | (FLAG_SPLIT_VIA_WORKSPACE if split_via_workspace else 0)
+             | (FLAG_SF_A_8X4 if sf_a_8x4 else 0))
     opts = _ws_opts(workspace, kernel, small_m_ctas, flags)
     _check("mxfp8_gemm", lib().mxfp8_gemm(a.data_ptr(), sf_a.data_ptr(), b.data_ptr(), sf_b.data_ptr(), m, n, k,
                                           c.data_ptr(), _ld(c, "c"), ctypes.byref(opts), _stream(stream)))

@@ -166,3 +166,30 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(binding.Fp8mmError):
         binding.lib()
+
+
+def test_sf8x4_layout_matches_header_formula():
+    """The small-M layout: 32-byte atoms of 8 rows x 4 K-blocks, atom (r8, g) at
+    (g * ceil(rows/8) + r8) * 32, byte (r % 8) * 4 + b % 4 inside; a bijection
+    onto [0, sf8x4_bytes) over the padded rows and blocks."""
+    for rows, k in [(1, 32), (5, 4096), (8, 160), (17, 14336), (64, 4128)]:
+        rows8 = -(-rows // 8) * 8
+        nb = -(-k // 128) * 4
+        assert fp8mm.sf8x4_bytes(rows, k) == rows8 * nb
+        seen = set()
+        for r in range(rows8):
+            for b in range(nb):
+                off = fp8mm.sf8x4_offset(rows, k, r, b)
+                atom = (b // 4) * (rows8 // 8) + r // 8
+                assert off == atom * 32 + (r % 8) * 4 + b % 4
+                seen.add(off)
+        assert seen == set(range(rows8 * nb))
+        assert fp8mm.sf8x4_offset(rows, k, rows8, 0) == -1 and fp8mm.sf8x4_offset(rows, k, 0, nb) == -1
+    assert fp8mm.sf8x4_bytes(0, 64) == 0
+
+
+def test_sf8x4_argument_errors_without_gpu():
+    L = binding.lib()
+    assert L.mxfp8_quantize_8x4(None, 4, 48, 48, None, 48, None, None) == 2      # k % 32
+    assert L.mxfp8_quantize_8x4(None, 4, 64, 64, None, 64, None, None) == 1      # null pointers
+    assert L.mxfp8_quantize_8x4(None, 0, 64, 64, None, 64, None, None) == 0      # nothing to do

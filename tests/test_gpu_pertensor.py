@@ -51,6 +51,27 @@ def test_tensor_scale_matches_the_oracle():
     assert s.item() == 1.0
 
 
+def test_tensor_scale_strided_and_repeated():
+    """A strided view (row stride 200, k 128: values past the view must not
+    count), rows spread over many blocks, and repeated calls on one output
+    word (each call starts from its own zeroed word)."""
+    import oracle as orc
+    base = synthetic.random_bf16((1000, 200), seed=8, sigma=3.0)
+    base[999, 100] = 5e3                                   # inside the view: the maximum
+    base[500, 190] = 1e6                                   # outside the view
+    view_d = gu.to_dev(base)[:, :128]
+    s_ref = orc.tensor_scale(synthetic.bits(base[:, :128].contiguous()))
+    out = torch.empty(1, dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        fp8mm.fp8_tensor_scale(view_d, out)
+        torch.cuda.synchronize()
+        assert np.float32(out.item()).view(np.uint32) == np.float32(s_ref).view(np.uint32)
+    big = synthetic.random_bf16((4096, 4096), seed=9)
+    big[4095, 4095] = -300.0
+    s, s_ref = _scale_both(big)
+    assert np.float32(s).view(np.uint32) == np.float32(s_ref).view(np.uint32)
+
+
 @pytest.mark.parametrize("scale", [1.0, 0.0078125, 3.0e-3, 1.7, 12345.0, 2.0 ** -85, 2.0 ** 127, 1.0e-30])
 def test_static_quantizer_every_bf16_value(scale):
     """All finite bf16 values at scales that keep the quotient in range, push
