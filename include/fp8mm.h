@@ -164,8 +164,8 @@ fp8mm_status fp8_gemm(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t
  *   stride ld_x elements), 1.0 for an all-zero tensor.
  * *scale is a device fp32 that the call overwrites (it is also the work word
  * of the reduction).  Requires k % 8 == 0, x 16-byte aligned, ld_x % 8 == 0,
- * rows * k / 8 < 2^32.  Three stream operations: a 4-byte memset and two
- * kernels.  rows == 0 or k == 0 writes 1.0. */
+ * rows * k / 8 < 2^32.  Three kernels on the stream (zero the word, fold
+ * the maximum into it, divide).  rows == 0 or k == 0 writes 1.0. */
 fp8mm_status fp8_tensor_scale(const void* x_bf16, int64_t rows, int64_t k, int64_t ld_x, float* scale,
                               void* stream);
 

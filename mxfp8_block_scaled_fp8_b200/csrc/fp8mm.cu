@@ -734,8 +734,8 @@ fp8mm_status fp8_tensor_scale(const void* x_bf16, int64_t rows, int64_t k, int64
   fp8mm_status st = current_device(&dev);
   if (st != FP8MM_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(scale, 0, sizeof(float), s);
-  if (e != cudaSuccess) return cuda_fail(e);
+  st = launch_pdl(tensor_scale_zero_kernel, dim3(1), dim3(1), 0, s, reinterpret_cast<unsigned*>(scale));
+  if (st != FP8MM_OK) return st;
   if (rows > 0 && k > 0) {
     // contiguous tensors are one flat run of vectors, strided ones go row by
     // row; at most eight blocks per SM

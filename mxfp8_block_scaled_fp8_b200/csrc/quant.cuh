@@ -210,8 +210,10 @@ __global__ void __launch_bounds__(kQ1Threads) quant_rowwise_2pass_kernel(const _
 // ------------------------------------------------------------------ per tensor
 
 // Per-tensor scale (page "FP8 推理基础设施（五）：从 DeepGEMM 到 vLLM", listing 3:
-// one scale per tensor, max|x| / 448), in two kernels after a zeroing memset
-// of the output word: every block takes the exact maximum of |x| over its
+// one scale per tensor, max|x| / 448), in three kernels chained by
+// programmatic dependent launch: one thread zeroes the output word (a kernel
+// rather than a memset, which cost ~3 us more between the neighbouring
+// kernels in a CUDA graph on B200), then every block takes the exact maximum of |x| over its
 // share (an unsigned 16-bit max over the sign-cleared bf16 bits, four 16-byte
 // loads in flight per thread: one flat run for a contiguous tensor, row by
 // row otherwise) and folds it into the word with one atomicMax (bf16 bits
@@ -265,6 +267,12 @@ __global__ void __launch_bounds__(kTensorThreads) tensor_amax_kernel(const __nv_
   m = max(m & 0xFFFFu, m >> 16) << 16;
   m = __reduce_max_sync(0xFFFFFFFFu, m);
   if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(word, m);
+}
+
+__global__ void tensor_scale_zero_kernel(unsigned* word) {
+  griddep_launch_dependents();
+  griddep_wait();  // the word may still be read by the preceding kernel
+  *word = 0u;
 }
 
 __global__ void tensor_scale_finalize_kernel(float* scale) {
