@@ -285,6 +285,20 @@ def _rows_measurements(fp8mm, synthetic, peaks, only=None):
         tf = 2.0 * 2048 * 1024 * 4096 / (t * 1e-3) / 1e12
         out["mxfp8_gemm_2048x1024x4096"] = {"ms": t, "TFLOPS": tf, "frac_fp8_peak": tf / fp8_peak}
 
+    if want("mxfp8_quantize_8192x8192"):
+        # MX quantizer on the step's activation shape, standalone (inside the
+        # step it follows the GEMM and shares HBM with the write-back of C)
+        x, _ = synthetic.ffn_up()
+        x = x.to(dev)
+        xs = [x] + [x.clone() for _ in range(_copies(x.numel() * 2) - 1)]
+        qx = torch.empty(x.shape, dtype=torch.uint8, device=dev)
+        sfx = torch.empty(fp8mm.sf_bytes(*x.shape), dtype=torch.uint8, device=dev)
+        t = _graph_time([lambda x_=x_: fp8mm.mxfp8_quantize(x_, qx, sfx) for x_ in xs])
+        R, Kq = x.shape
+        gbs = (3.0 * R * Kq + R * Kq / 32) / (t * 1e-3) / 1e9
+        out["mxfp8_quantize_8192x8192"] = {"ms": t, "GB/s": gbs, "frac_hbm": gbs / hbm}
+        del x, xs, qx, sfx
+
     if want("mxfp8_quantize_22016x8192"):
         # MX quantizer on the FFN weight (done once at load), standalone
         _, w = synthetic.ffn_up()
