@@ -359,6 +359,24 @@ def _rows_measurements(fp8mm, synthetic, peaks, only=None):
     return out
 
 
+def _rows_summary(rows):
+    """The per-row roofline fractions at a glance: each quantizer and GEMM row's
+    fraction, and the decode sweep's range per way of calling it."""
+    out = {}
+    for name, r in rows.items():
+        if isinstance(r, dict) and "frac_hbm" in r:
+            out[name] = {"frac_hbm": r["frac_hbm"]}
+        elif isinstance(r, dict) and "frac_fp8_peak" in r:
+            out[name] = {"frac_fp8_peak": r["frac_fp8_peak"]}
+    dec = rows.get("decode")
+    if dec:
+        for key, label in (("gemm_frac_hbm", "decode_gemm_alone"), ("frac_hbm", "decode_quantize_then_gemm"),
+                           ("fused_frac_hbm", "decode_quantize_gemm")):
+            v = [c[key] for c in dec.values()]
+            out[label] = {"frac_hbm_min": min(v), "frac_hbm_max": max(v), "cases": len(v)}
+    return out
+
+
 def _sustained(step, gemm, stream, local, pci, seconds: float = 3.0, k: int = 100):
     """The headline step back to back for `seconds` (the GPU settles at its
     power cap); then k more steps and k GEMM calls, each timed alone with CUDA
@@ -599,6 +617,7 @@ def run_ours(args):
             line["cpu_baseline"]["per_config"] = cpu_per_config()
     if rows is not None:
         line["rows"] = rows
+        line["rows_summary"] = _rows_summary(rows)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:

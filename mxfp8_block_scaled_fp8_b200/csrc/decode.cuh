@@ -196,9 +196,17 @@ __device__ __forceinline__ void cluster_reduce_slice(const float* red, int rank,
       const float o[4] = {sum.x, sum.y, sum.z, sum.w};
       const int n0 = t * 128 + quad * 4;
       __nv_bfloat16* dst = p.c + static_cast<int64_t>(j) * p.ldc + n0;
+      if (n0 + 4 <= p.n && (reinterpret_cast<uintptr_t>(dst) & 7u) == 0) {
+        // four outputs in one 8-byte store (a warp writes 256 contiguous bytes)
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
+        *reinterpret_cast<uint2*>(dst) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+      } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (n0 + e < p.n) dst[e] = __float2bfloat16_rn(o[e]);
+        for (int e = 0; e < 4; ++e)
+          if (n0 + e < p.n) dst[e] = __float2bfloat16_rn(o[e]);
+      }
     }
   }
 }

@@ -47,3 +47,16 @@ def test_percentiles_nearest_rank():
     assert bench.percentiles([]) is None
     q = bench.percentiles([3.0])
     assert q["p10"] == q["p50"] == q["p90"] == 3.0
+
+
+def test_rows_summary_ranges():
+    rows = {"quantize_rowwise_8192x8192": {"ms": 1.0, "GB/s": 5.0, "frac_hbm": 0.9},
+            "fp8_gemm_8192x2048x8192": {"ms": 1.0, "TFLOPS": 2.0, "frac_fp8_peak": 0.8},
+            "decode": {"a": {"gemm_frac_hbm": 0.5, "frac_hbm": 0.4, "fused_frac_hbm": 0.45},
+                       "b": {"gemm_frac_hbm": 0.7, "frac_hbm": 0.6, "fused_frac_hbm": 0.65}},
+            "timing": "x"}
+    s = bench._rows_summary(rows)
+    assert s["quantize_rowwise_8192x8192"] == {"frac_hbm": 0.9}
+    assert s["fp8_gemm_8192x2048x8192"] == {"frac_fp8_peak": 0.8}
+    assert s["decode_gemm_alone"] == {"frac_hbm_min": 0.5, "frac_hbm_max": 0.7, "cases": 2}
+    assert s["decode_quantize_gemm"]["frac_hbm_min"] == 0.45
