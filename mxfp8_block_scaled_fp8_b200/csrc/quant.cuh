@@ -427,4 +427,73 @@ __global__ void __launch_bounds__(kQ2Threads) quant_mx_kernel(const __nv_bfloat1
   }
 }
 
+// Activations of at most 128 rows (one row tile; the launcher uses it for
+// decode activations of up to 32 rows with a long K): one warp per (scale
+// line L, segment of 32 K blocks).  Line L of a 512-byte
+// chunk holds the words of rows L, L + 32, L + 64 and L + 96, so the warp
+// quantizes those of its rows that exist -- lane l owns block 32 seg + l of
+// each, with every row's four loads in flight at once -- and writes the whole
+// 16-byte line (zero words for rows past the last).  32 x segments warps
+// instead of 128 x segments, none of them for padding rows only, and the same
+// codes, exponents and padding bytes as quant_mx_kernel.
+__global__ void __launch_bounds__(kQ2Threads) quant_mx_lines_kernel(const __nv_bfloat16* __restrict__ x, int rows,
+                                                                    int64_t k, int64_t ld_x, uint8_t* __restrict__ q,
+                                                                    int64_t ld_q, uint8_t* __restrict__ sf, int n_kc) {
+  const int lane = threadIdx.x & 31;
+  const int nkb = static_cast<int>(k / 32);
+  const int nkb4 = n_kc * 4;
+  const int segs = (nkb4 + 31) / 32;
+  const int task = blockIdx.x * (kQ2Threads / 32) + (threadIdx.x >> 5);
+  const int L = task % 32, seg = task / 32;
+  const bool q16 = (reinterpret_cast<uintptr_t>(q) % 16 == 0) && (ld_q % 16 == 0);
+  griddep_launch_dependents();  // a following GEMM may start prefetching its weights
+  griddep_wait();               // x and the outputs may belong to the preceding kernel
+  if (seg >= segs) return;
+  const int kb = seg * 32 + lane;
+  uint4 v[4][4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const int row = L + 32 * g;
+    const bool real = row < rows && kb < nkb;
+    const __nv_bfloat16* src = x + static_cast<int64_t>(real ? row : 0) * ld_x + static_cast<int64_t>(kb) * 32;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) v[g][t] = real ? ld_stream_16(src + 8 * t) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  uint32_t word[4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const int row = L + 32 * g;
+    const bool real = row < rows && kb < nkb;
+    const int e = real ? mx_exponent(bf16x32_absmax(v[g])) : 0;
+    if (real) {
+      const float inv = mx_inv_scale(e);  // exact: power-of-two scaling
+      uint2 c[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        float f[8];
+        bf16x8_to_f32(v[g][t], f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) f[u] *= inv;
+        c[t] = f32x8_to_e4m3(f);
+      }
+      uint8_t* dst = q + static_cast<int64_t>(row) * ld_q + static_cast<int64_t>(kb) * 32;
+      if (q16) {
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
+        reinterpret_cast<uint4*>(dst)[1] = make_uint4(c[2].x, c[2].y, c[3].x, c[3].y);
+      } else {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) reinterpret_cast<uint2*>(dst)[t] = c[t];
+      }
+    }
+    // the word of blocks kb..kb+3 of this row (lanes L..L+3, L % 4 == 0)
+    const uint32_t e1 = __shfl_down_sync(0xFFFFFFFFu, static_cast<uint32_t>(e), 1);
+    const uint32_t e2 = __shfl_down_sync(0xFFFFFFFFu, static_cast<uint32_t>(e), 2);
+    const uint32_t e3 = __shfl_down_sync(0xFFFFFFFFu, static_cast<uint32_t>(e), 3);
+    word[g] = static_cast<uint32_t>(e) | (e1 << 8) | (e2 << 16) | (e3 << 24);
+  }
+  if ((lane & 3) == 0 && kb < nkb4)
+    *reinterpret_cast<uint4*>(sf + static_cast<int64_t>(kb / 4) * 512 + L * 16) =
+        make_uint4(word[0], word[1], word[2], word[3]);
+}
+
 }  // namespace fp8mm

@@ -116,7 +116,9 @@ def _edge_tensor():
     return x
 
 
-@pytest.mark.parametrize("rows,k", [(1, 512), (200, 96), (129, 4096), (3, 32), (64, 14336)])
+@pytest.mark.parametrize("rows,k", [(1, 512), (200, 96), (129, 4096), (3, 32), (64, 14336),
+                                    # few rows and a long K: the one-warp-per-scale-line kernel
+                                    (1, 8192), (17, 8224), (32, 14336), (5, 9984)])
 def test_mx_ragged_and_small(rows, k):
     import oracle as orc
     _assert_mx(orc, synthetic.random_bf16((rows, k), seed=rows + k), f"mx {rows}x{k}")
@@ -210,3 +212,18 @@ def test_bad_arguments_are_rejected():
     x = torch.zeros((4, 12), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(fp8mm.Fp8mmError):
         fp8mm.fp8_quantize_rowwise(x)                   # k % 8 != 0
+
+
+def test_mx_few_rows_long_k_strided_and_unaligned_q():
+    """The one-warp-per-scale-line kernel (few rows, long K) on a strided
+    input and an output whose rows are only 8-byte aligned."""
+    import oracle as orc
+    base = synthetic.random_bf16((20, 8704), seed=15, sigma=4.0)
+    base[3, 100:200] = 0.0
+    view = base[:, :8192]
+    q_ref, sf_ref = orc.mx_quantize(synthetic.bits(view.contiguous()))
+    qbuf = torch.zeros((20, 8200), dtype=torch.uint8, device="cuda")   # row stride 8200: 8-byte aligned rows
+    q, sf = fp8mm.mxfp8_quantize(gu.to_dev(base)[:, :8192], q=qbuf[:, :8192])
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(sf.cpu().numpy(), gu.sf_layout_from_canonical(sf_ref, 20, 8192))
