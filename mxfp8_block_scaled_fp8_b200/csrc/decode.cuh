@@ -89,10 +89,12 @@ struct DecodeCfg {
   static constexpr int kQuantWarps = kQX ? 2 : (kSF8 ? 1 : 0);
   static constexpr int kThreads = 192 + 32 * kQuantWarps;
   static constexpr int kQuantWarp0 = 6;
-  // Token tiles up to 32 keep shared memory and registers within half an SM,
-  // so the next kernel on the stream (launched early, programmatically) can
-  // hold a CTA on each SM and start streaming while this one finishes.
-  static constexpr int kMinBlocksPerSm = kNM <= 32 ? 2 : 1;
+  // Shared memory and registers within half an SM, so two CTAs share an SM
+  // and the next kernel on the stream (launched early, programmatically) can
+  // hold a CTA on each SM and start streaming while this one finishes.  (The
+  // 8x4-scale variant with 48/64-token tiles keeps one per SM: its extra warp
+  // would not fit the registers.)
+  static constexpr int kMinBlocksPerSm = (kNM <= 32 || !kSF8) ? 2 : 1;
   static constexpr int kWBytes = 128 * 128;
   static constexpr int kXBytes = kNM * 128;
   static_assert(!kQX || kNM == 16, "activation quantized in the kernel for m <= 8 (16-token tile)");

@@ -187,11 +187,11 @@ using G1 = GemmCfg<false, 256, 4, 2>;
 using G2 = GemmCfg<true, 256, 4, 1>;
 using G1n = GemmCfg<false, 128, 6, 2>;  // 128 x 128 tiles
 using G2n = GemmCfg<true, 128, 6, 2>;
-// Small-M ring depth: as many stages as shared memory holds (the weight
-// stream needs ~25 MB in flight GPU-wide to cover the loaded HBM latency).
-// Stages of the small-M kernel: token tiles up to 32 run two CTAs per SM
-// (half the shared memory each), larger ones one CTA with a deeper ring.
-constexpr int dec_stages(int nm) { return nm <= 16 ? 5 : nm <= 32 ? 5 : nm <= 48 ? 9 : 8; }
+// Small-M ring depth: as many stages as half an SM's shared memory holds, so
+// that two CTAs share each SM.  For 48- and 64-token tiles that is 4 stages
+// (one CTA per SM with 9 / 8 stages was 6-16 % slower on the decode shapes at
+// m = 33..64, level on down-projection m = 64).
+constexpr int dec_stages(int nm) { return nm <= 32 ? 5 : 4; }
 // With the activation quantized in the kernel (m <= 8).
 constexpr int dec_stages_qx(int nm) { return nm <= 16 ? 5 : 0; }
 
@@ -508,17 +508,18 @@ static int small_m_l2_ahead(int64_t units, int64_t ctas, int64_t sms) {
 }
 
 // CTAs of the small-M kernel: the requested number; else one per SM, or two
-// per SM when two fit (token tiles up to 32), the weight tiles are short
-// (<= 48 K slabs, so the finer split adds at most about one contributor per
-// tile) and every CTA keeps >= 8 slabs; in every case no fewer than 4 slabs
-// per CTA, never more CTAs than slabs, never fewer than the tiles.
+// per SM when the weight tiles are short (<= 48 K slabs, so the finer split
+// adds at most about one contributor per tile) and every CTA keeps >= 8
+// slabs; in every case no fewer than 4 slabs per CTA, never more CTAs than
+// slabs, never fewer than the tiles.
 //
 // That count is replaced by a tile-aligned one -- s CTAs per weight tile,
 // with s dividing the tile's K slabs, so every CTA runs one segment inside
-// one tile and all contributors of a tile are equal -- when the largest such
-// count that fits the SMs (two per SM for token tiles up to 32) comes within
-// 80 % of it (16-token tiles) or 60 % (larger tiles, whose split-tile partials
-// cost more).  Measured on B200 with back-to-back calls (GEMM alone): 6144 x
+// one tile and all contributors of a tile are equal (and reduce inside a
+// cluster) -- when the largest such count that fits two CTAs per SM comes
+// within 80 % of it (16-token tiles) or 60 % (larger tiles, whose split-tile
+// partials cost more).  Measured on B200 with back-to-back calls (GEMM alone,
+// before 48- and 64-token tiles ran two per SM): 6144 x
 // 4096 at m <= 32 with 192 CTAs instead of 148 is 12-17 % faster and at m = 64
 // with 96 instead of 148 10 %, 4096 x 14336 at m <= 8 with 256 instead of 148
 // 8 % and at m = 64 with 128 instead of 148 6 %, 14336 x 4096 at m = 32 with
@@ -537,9 +538,9 @@ static int64_t best_cluster_ctas(int64_t n_tiles, int64_t num_k, int64_t slots) 
 static int small_m_ctas(int64_t units, int64_t n_tiles, int64_t num_k, int nm, int64_t requested, int64_t sms) {
   int64_t g = requested;
   if (g <= 0) {
-    const bool two_per_sm = nm <= 32 && num_k <= 48 && units >= 2 * sms * 8;
+    const bool two_per_sm = num_k <= 48 && units >= 2 * sms * 8;
     g = std::min<int64_t>(two_per_sm ? 2 * sms : sms, std::max<int64_t>(n_tiles, cdiv(units, kMinSlabsPerCta)));
-    const int64_t slots = nm <= 32 ? 2 * sms : sms;
+    const int64_t slots = 2 * sms;
     int64_t aligned = 0;
     for (int64_t s = 1; s <= num_k / kMinSlabsPerCta; ++s)
       if (num_k % s == 0 && n_tiles * s <= slots) aligned = n_tiles * s;
@@ -584,7 +585,7 @@ static fp8mm_status launch_small_m(const void* a, const uint8_t* sfa, const void
       // No workspace: a tile-aligned split reduced in clusters where one
       // fits (automatic count only), else one CTA per weight tile over all
       // of K (no partial sums).
-      const int64_t g = (requested > 0 || via_ws) ? 0 : best_cluster_ctas(p.n_tiles, p.num_k, dev.sms * (nm <= 32 ? 2 : 1));
+      const int64_t g = (requested > 0 || via_ws) ? 0 : best_cluster_ctas(p.n_tiles, p.num_k, 2 * dev.sms);
       p.ctas = static_cast<int>(g > 0 ? g : p.n_tiles);
       p.cluster_s = g > 0 ? cluster_split(g, p.n_tiles, p.num_k) : 0;
     }

@@ -122,9 +122,9 @@ def test_workspace_sizes():
         nm = 16 if m <= 16 else 32 if m <= 32 else 48 if m <= 48 else 64
         tickets = -(-(-(-n // 128) * 4) // 256) * 256
         return (fp8mm.workspace_bytes(m, n, k) - tickets) // (2 * 128 * nm * 4)
-    expected = {(1, 14336, 4096): 296, (8, 14336, 4096): 296, (32, 14336, 4096): 224, (64, 14336, 4096): 112,
-                (1, 4096, 14336): 256, (8, 4096, 14336): 256, (32, 4096, 14336): 256, (64, 4096, 14336): 128,
-                (1, 6144, 4096): 192, (8, 6144, 4096): 192, (32, 6144, 4096): 192, (64, 6144, 4096): 96,
+    expected = {(1, 14336, 4096): 296, (8, 14336, 4096): 296, (32, 14336, 4096): 224, (64, 14336, 4096): 224,
+                (1, 4096, 14336): 256, (8, 4096, 14336): 256, (32, 4096, 14336): 256, (64, 4096, 14336): 256,
+                (1, 6144, 4096): 192, (8, 6144, 4096): 192, (32, 6144, 4096): 192, (64, 6144, 4096): 192,
                 (8, 1024, 2048): 32, (3, 200, 96): 2}
     got = {shape: auto_ctas(*shape) for shape in expected}
     assert got == expected
