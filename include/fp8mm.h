@@ -69,9 +69,11 @@ typedef struct fp8mm_opts {
   /* Device scratch for split K: fp32 partial tiles plus 32-bit arrival
    * counters, fp8mm_workspace_bytes(m, n, k, small_m_ctas) bytes, 256-byte
    * aligned.  Used by the small-M kernel (mxfp8_gemm, m <= 64) and, for
-   * m > 64, by the paired-SM kernel where its 256 x 256 tiles fill less than
-   * one wave of SM pairs (the K range of each tile is then split over several
-   * pairs; fp8mm_workspace_bytes is 0 for shapes that are not split).
+   * m > 64 and K >= 8192, by the paired-SM kernel: the 256 x 256 tiles of its
+   * last, partly filled wave of SM pairs (all tiles, where they fill less than
+   * one wave) have their K range split over several pairs, so that the wave
+   * keeps every pair busy (fp8mm_workspace_bytes is 0 for shapes that are
+   * never split).
    * Caller-owned.  It must be zeroed once before first use (e.g.
    * cudaMemsetAsync); every successful call leaves the counters zero again.
    * After a call that reported FP8MM_ERR_DEVICE it must be zeroed again.
@@ -150,8 +152,8 @@ fp8mm_status fp8_quantize_rowwise(const void* x_bf16, int64_t rows, int64_t k, i
  * Requires k % 16 == 0, a/b 16-byte aligned, c 2-byte aligned, ldc >= n (rows
  * whose address is 16-byte aligned are written with 16-byte stores).
  * m == 0 or n == 0 is a no-op; k == 0 writes zeros.  opt may be NULL; with
- * opt->workspace, m > 64 shapes that fill less than one wave of SM pairs split
- * K over the pairs (see fp8mm_opts.workspace). */
+ * opt->workspace, m > 64 shapes split the K range of the tiles of their last
+ * wave of SM pairs over the pairs (see fp8mm_opts.workspace). */
 fp8mm_status fp8_gemm(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t n, int64_t k,
                       const float* scale_a, const float* scale_b, void* c_bf16, int64_t ldc,
                       const fp8mm_opts* opt, void* stream);
@@ -251,8 +253,9 @@ fp8mm_status mxfp8_quantize_8x4(const void* x_bf16, int64_t rows, int64_t k, int
  * 128-row side, tokens the N side, and K is split stream-K style over the SMs
  * when opt->workspace is given (see fp8mm_workspace_bytes); partial sums are
  * reduced deterministically (fixed order) by the last CTA of each tile.  With
- * m > 64 and a workspace, shapes whose 256 x 256 tiles fill less than one
- * wave of SM pairs split each tile's K range over pairs the same way. */
+ * m > 64 and a workspace, the 256 x 256 tiles of the last, partly filled
+ * wave of SM pairs (all tiles, where they fill less than one wave) split
+ * their K range over pairs the same way. */
 fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e4m3, const uint8_t* sf_b,
                         int64_t m, int64_t n, int64_t k, void* c_bf16, int64_t ldc, const fp8mm_opts* opt,
                         void* stream);
@@ -285,9 +288,21 @@ size_t fp8mm_quantize_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k, int3
 
 /* Workspace bytes a GEMM of this shape uses: for m <= 64 those of the
  * small-M kernel with `ctas` CTAs (0 = its automatic choice); for m > 64 those
- * of the paired-SM kernel's K split (`ctas` ignored), 0 when the shape is not
- * split.  The current device's SM count decides; on a host without a GPU, 148. */
+ * of the paired-SM kernel's K split (`ctas` ignored): room for one split part
+ * per SM pair, (SMs / 2) x 256 KiB of partials plus the counters, whatever
+ * the tile count, for K >= 8192, and 0 below (never split).  The current
+ * device's SM count decides; on a host without a GPU, 148. */
 size_t fp8mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas);
+
+/* The paired-SM kernel's K split for an m > 64 call with a workspace when
+ * `pairs` SM pairs run at once: returns the K parts of each split tile (1: no
+ * split) and stores in *dp_tiles (if not NULL) how many of the ceil(m/256) x
+ * ceil(n/256) tiles, taken in raster order, run whole; the rest, the last
+ * partly filled wave, are split.  Parts: the most that fit the pairs that
+ * wave leaves, each of at least 16 K slabs of 128, at most 8; none for
+ * m <= 64, K < 8192, or tiles that fill whole waves.  Host-only; a planning
+ * query with no device work (invalid sizes give 1 and 0). */
+int32_t fp8mm_pair_split_plan(int64_t m, int64_t n, int64_t k, int32_t pairs, int32_t* dp_tiles);
 
 /* ---------------------------------------------------------------- KV cache */
 

@@ -22,8 +22,9 @@ Typical use (all tensors on the current CUDA device, the current stream)::
     c = fp8mm.mxfp8_quantize_gemm(x_bf16, qw, sfw, workspace=ws, weights_ready=True)
 
 ``workspace_bytes`` also sizes the workspace that lets long-K GEMMs with
-m > 64 and few output tiles split K over SM pairs (0 when a shape does not
-split); ``sf_to_canonical`` / ``sf_from_canonical`` convert scales to and
+m > 64 split the K range of the tiles of their last, partly filled wave over
+SM pairs (0 when a shape never splits; ``pair_split_plan`` tells how a shape
+splits); ``sf_to_canonical`` / ``sf_from_canonical`` convert scales to and
 from the row-major [rows, k / 32] tensor.  For activations of a few token
 rows, ``mxfp8_quantize_8x4`` writes the scales in the small-M layout (rows
 padded to 8 instead of 128) that ``mxfp8_gemm(..., sf_a_8x4=True)`` reads.
@@ -33,5 +34,5 @@ from .fp8mm import (  # noqa: F401
     fp8_quantize_static, fp8_tensor_scale, last_device_error,
     mxfp8_gemm, mxfp8_quantize, mxfp8_quantize_8x4, mxfp8_quantize_gemm, selftest_wait_timeout, sf_bytes,
     sf_from_canonical, sf_offset, sf_to_canonical, sf8x4_bytes, sf8x4_offset,
-    quantize_gemm_workspace_bytes, version, workspace_bytes,
+    pair_split_plan, quantize_gemm_workspace_bytes, version, workspace_bytes,
 )

@@ -279,7 +279,9 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX, kSF8>::kThreads,
     // kb).  When the caller vouches that the weights do not depend on the
     // preceding kernel (prefetch_w), the weights of the first stages are
     // requested before griddepcontrol.wait; the activation always after it.
-    if (lane == 0) {
+    // The whole warp runs the loops; one elected lane issues (see
+    // elect_one_sync).
+    {
       if (!p.prefetch_w) griddep_wait();
       const int64_t nslabs = u_end - u_begin;
       const int npre = static_cast<int>(nslabs < kStages ? nslabs : kStages);
@@ -290,9 +292,13 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX, kSF8>::kThreads,
                                       : Cfg::kWBytes + Cfg::kXBytes + 1024u;
       int t = t0, kb = kb0;
       for (int i = 0; i < npre; ++i) {  // fresh stages: nothing to wait for
-        mbar_arrive_expect_tx(&full[i], kTx);
-        tma_load_2d(smem + Cfg::kOffW + i * Cfg::kWBytes, &tmW, &full[i], kb * 128, t * 128);
-        bulk_load(smem + Cfg::kOffSfw + i * 512, p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u, &full[i]);
+        if (elect_one_sync()) {
+          mbar_arrive_expect_tx(&full[i], kTx);
+          tma_load_2d(smem + Cfg::kOffW + i * Cfg::kWBytes, &tmW, &full[i], kb * 128, t * 128);
+          bulk_load(smem + Cfg::kOffSfw + i * 512, p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u,
+                    &full[i]);
+        }
+        __syncwarp();
         if (++kb == p.num_k) {
           kb = 0;
           ++t;
@@ -303,8 +309,11 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX, kSF8>::kThreads,
       // programmatic launch, for the preceding kernel).
       const int64_t l2_end = npre + p.l2_ahead < nslabs ? npre + p.l2_ahead : nslabs;
       for (int64_t i = npre; i < l2_end; ++i) {
-        tma_prefetch_l2_2d(&tmW, kb * 128, t * 128);
-        bulk_prefetch_l2(p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u);
+        if (elect_one_sync()) {
+          tma_prefetch_l2_2d(&tmW, kb * 128, t * 128);
+          bulk_prefetch_l2(p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u);
+        }
+        __syncwarp();
         if (++kb == p.num_k) {
           kb = 0;
           ++t;
@@ -315,9 +324,12 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX, kSF8>::kThreads,
       kb = kb0;
       for (int i = 0; i < npre; ++i) {
         if (!kQX) {
-          tma_load_2d(smem + Cfg::kOffX + i * Cfg::kXBytes, &tmX, &full[i], kb * 128, 0);
-          if (!kSF8)
-            bulk_load(smem + Cfg::kOffSfx + i * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[i]);
+          if (elect_one_sync()) {
+            tma_load_2d(smem + Cfg::kOffX + i * Cfg::kXBytes, &tmX, &full[i], kb * 128, 0);
+            if (!kSF8)
+              bulk_load(smem + Cfg::kOffSfx + i * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u, &full[i]);
+          }
+          __syncwarp();
         }
         if (++kb == p.num_k) {
           kb = 0;
@@ -329,17 +341,20 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX, kSF8>::kThreads,
       uint32_t issued_mask = (npre == kStages) ? ((1u << kStages) - 1u) : ((1u << npre) - 1u);
       uint32_t issued_parity = 0;
       for (int64_t i = npre; i < nslabs; ++i) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) break;
-        mbar_arrive_expect_tx(&full[stage], kTx);
-        tma_load_2d(smem + Cfg::kOffW + stage * Cfg::kWBytes, &tmW, &full[stage], kb * 128, t * 128);
-        bulk_load(smem + Cfg::kOffSfw + stage * 512, p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u,
-                  &full[stage]);
-        if (!kQX) {
-          tma_load_2d(smem + Cfg::kOffX + stage * Cfg::kXBytes, &tmX, &full[stage], kb * 128, 0);
-          if (!kSF8)
-            bulk_load(smem + Cfg::kOffSfx + stage * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u,
-                      &full[stage]);
+        if (!warp_wait(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) break;
+        if (elect_one_sync()) {
+          mbar_arrive_expect_tx(&full[stage], kTx);
+          tma_load_2d(smem + Cfg::kOffW + stage * Cfg::kWBytes, &tmW, &full[stage], kb * 128, t * 128);
+          bulk_load(smem + Cfg::kOffSfw + stage * 512, p.sfw + (static_cast<int64_t>(t) * p.n_kc + kb) * 512, 512u,
+                    &full[stage]);
+          if (!kQX) {
+            tma_load_2d(smem + Cfg::kOffX + stage * Cfg::kXBytes, &tmX, &full[stage], kb * 128, 0);
+            if (!kSF8)
+              bulk_load(smem + Cfg::kOffSfx + stage * 512, p.sfx + static_cast<int64_t>(kb) * 512, 512u,
+                        &full[stage]);
+          }
         }
+        __syncwarp();
         issued_mask |= 1u << stage;
         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == kStages) {
@@ -358,47 +373,53 @@ __global__ void __launch_bounds__(DecodeCfg<kNM, kStages, kQX, kSF8>::kThreads,
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues (see elect_one_sync).
+    {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int64_t u = u_begin; ok && u < u_end;) {
         const int kb0 = static_cast<int>(u % p.num_k);
         const int kb1 = static_cast<int>(kb0 + (u_end - u) < p.num_k ? kb0 + (u_end - u) : p.num_k);
-        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, kSiteMmaAccEmpty)) break;
+        if (!warp_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, kSiteMmaAccEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kNM);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag, kSiteMmaFull)) {
+          if (!warp_wait(&full[stage], phase, p.timeout_ns, abort_flag, kSiteMmaFull)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sfw_t = tmem_base + static_cast<uint32_t>(Cfg::kSfCol0 + stage * 8);
-          const uint32_t sfx_t = sfw_t + 4u;
-          tmem_cp_32x128b_warpx4(sfw_t, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfw + stage * 512)));
-          tmem_cp_32x128b_warpx4(sfx_t, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfx + stage * 512)));
-          const uint64_t wdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffW + stage * Cfg::kWBytes));
-          const uint64_t xdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffX + stage * Cfg::kXBytes));
+          if (elect_one_sync()) {
+            const uint32_t sfw_t = tmem_base + static_cast<uint32_t>(Cfg::kSfCol0 + stage * 8);
+            const uint32_t sfx_t = sfw_t + 4u;
+            tmem_cp_32x128b_warpx4(sfw_t, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfw + stage * 512)));
+            tmem_cp_32x128b_warpx4(sfx_t, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfx + stage * 512)));
+            const uint64_t wdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffW + stage * Cfg::kWBytes));
+            const uint64_t xdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffX + stage * Cfg::kXBytes));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_mxf8f6f4(d_tmem, wdesc + 2u * kk, xdesc + 2u * kk, idesc_mxf8f6f4(128, kNM, kk, kk), sfw_t, sfx_t,
-                         (kb != kb0) || (kk != 0));
-          tc_commit(&empty[stage]);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_mxf8f6f4(d_tmem, wdesc + 2u * kk, xdesc + 2u * kk, idesc_mxf8f6f4(128, kNM, kk, kk), sfw_t, sfx_t,
+                           (kb != kb0) || (kk != 0));
+            tc_commit(&empty[stage]);
+          }
+          __syncwarp();
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(&acc_full[acc]);
+        if (elect_one_sync()) tc_commit(&acc_full[acc]);
+        __syncwarp();
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
         u += kb1 - kb0;
       }
-      tc_commit(drain);
+      if (elect_one_sync()) tc_commit(drain);
+      __syncwarp();
       mbar_wait(drain, 0, p.timeout_ns, nullptr, kSiteDrain);
     }
     __syncwarp();

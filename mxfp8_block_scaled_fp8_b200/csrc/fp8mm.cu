@@ -326,52 +326,76 @@ static fp8mm_status max_pairs(const void* kern, int smem, int threads, const Dev
 // 8192 x 2048 x 8192 (B 16 MB, L2-resident) 16 are 1.6 % slower than 8.
 static int pair_group_m(int64_t n, int64_t k) { return n * k > (int64_t{64} << 20) ? 2 * kPairGroupM : kPairGroupM; }
 
-// K parts per tile of the paired-SM kernel (split K): where its 256 x 256
-// tiles fill less than one wave of SM pairs and K has at least 64 slabs of
-// 128, the most parts that still fit in one wave, each of at least 16 slabs,
-// at most 8; else 1.  Only for m > 64 (below that mxfp8_gemm runs the
-// small-M kernel).  The fp32 partials cost a write and a read of 256 KB per
-// part and tile through L2, so short K gains nothing: measured on B200,
-// 512 x 2048 x 8192 (16 tiles, 4 parts of 16 slabs) takes 23.2 us against
-// 29.5 us unsplit (MX), but 2048 x 1024 x 4096 with 2 parts of 16 slabs 21.4
-// us against 18.3 us on 128 x 128 single-SM tiles.
-static int pair_split(int64_t m, int64_t n, int64_t k, int64_t sms) {
+// Split K of the paired-SM kernel over `pairs` co-resident SM pairs: the
+// tiles of the last, partly filled wave (all tiles, where they fill less
+// than one wave) run as `split` K parts each -- the most parts that still fit
+// in that wave, each of at least 16 slabs of 128, at most 8 -- so that the
+// wave keeps every pair busy; the other tiles run whole.  Only for m > 64
+// (below that mxfp8_gemm runs the small-M kernel) and K of at least 64 slabs:
+// the fp32 partials cost a write and a read of 256 KB per part and tile
+// through L2, so short K gains nothing.  Measured on B200: 512 x 2048 x 8192
+// (16 tiles, 4 parts of 16 slabs) takes 23.2 us against 29.5 us unsplit
+// (MX), but 2048 x 1024 x 4096 with 2 parts of 16 slabs 21.4 us against 18.3
+// us on 128 x 128 single-SM tiles.
+struct PairPlan {
+  int split;     // K parts per split tile (1: no split)
+  int dp_tiles;  // tiles run whole; the rest are split
+};
+static PairPlan pair_plan(int64_t m, int64_t n, int64_t k, int64_t pairs) {
   const int64_t num_k = cdiv(k, kBK);
-  if (m <= 64 || num_k < 64) return 1;
   const int64_t tiles = cdiv(m, 256) * cdiv(n, 256);
-  const int64_t pairs = std::max<int64_t>(1, sms / 2);
-  const int64_t s = std::min<int64_t>(std::min<int64_t>(pairs / tiles, num_k / 16), 8);
-  return static_cast<int>(std::max<int64_t>(1, s));
+  if (m <= 64 || num_k < 64 || pairs < 2) return {1, static_cast<int>(tiles)};
+  const int64_t rem = tiles % pairs;
+  if (rem == 0) return {1, static_cast<int>(tiles)};
+  const int64_t s = std::min<int64_t>(std::min<int64_t>(pairs / rem, num_k / 16), 8);
+  if (s < 2) return {1, static_cast<int>(tiles)};
+  return {static_cast<int>(s), static_cast<int>(tiles - rem)};
 }
 static size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
-// Workspace of a split-K paired launch: the partials, then the counters.
-static size_t pair_partials_bytes(int64_t m, int64_t n, int split) {
-  return round256(static_cast<size_t>(cdiv(m, 256) * cdiv(n, 256)) * split * 2 * kPairPartFloats * sizeof(float));
+// Workspace of a split paired launch on a device with `sms` SMs: at most one
+// split part per co-resident pair (<= sms / 2), each with both CTAs'
+// partials, then one arrival counter per (split tile, rank).  Shapes the plan
+// never splits need none.
+static size_t pair_partials_bytes(int64_t sms) {
+  return round256(static_cast<size_t>(std::max<int64_t>(1, sms / 2)) * 2 * kPairPartFloats * sizeof(float));
 }
-static size_t pair_split_bytes(int64_t m, int64_t n, int split) {
-  if (split <= 1) return 0;
-  return pair_partials_bytes(m, n, split) + round256(static_cast<size_t>(cdiv(m, 256) * cdiv(n, 256)) * 2 * 4);
+static size_t pair_split_bytes(int64_t m, int64_t k, int64_t sms) {
+  if (m <= 64 || cdiv(k, kBK) < 64) return 0;
+  return pair_partials_bytes(sms) + round256(static_cast<size_t>(std::max<int64_t>(1, sms / 2)) * 2 * 4);
 }
-// Split for a tiled call: > 1 when a workspace is given, the kernel choice
-// allows the paired kernel (AUTO, TILED, TILED_2SM) and the shape is split;
-// -1 when that workspace is too small or misaligned.
+// Whether a tiled call may split: a workspace is given and the kernel choice
+// allows the paired kernel (AUTO, TILED, TILED_2SM); 1 if so, 0 if not, -1
+// when the shape may split and that workspace is too small or misaligned.
 static int tiled_split(const fp8mm_opts* opt, int kind, int64_t m, int64_t n, int64_t k, int64_t sms) {
-  if (opt == nullptr || opt->workspace == nullptr) return 1;
-  if (kind != FP8MM_KERNEL_AUTO && kind != FP8MM_KERNEL_TILED && kind != FP8MM_KERNEL_TILED_2SM) return 1;
-  const int s = pair_split(m, n, k, sms);
-  if (s <= 1) return 1;
-  if (opt->workspace_bytes < pair_split_bytes(m, n, s) || !aligned(opt->workspace, 256)) return -1;
-  return s;
+  (void)n;
+  if (opt == nullptr || opt->workspace == nullptr) return 0;
+  if (kind != FP8MM_KERNEL_AUTO && kind != FP8MM_KERNEL_TILED && kind != FP8MM_KERNEL_TILED_2SM) return 0;
+  const size_t need = pair_split_bytes(m, k, sms);
+  if (need == 0) return 0;
+  if (opt->workspace_bytes < need || !aligned(opt->workspace, 256)) return -1;
+  return 1;
+}
+// Tiled kernel of a call that has passed tiled_split (ws: a usable
+// workspace): tiled_kind's choice, except that a shape whose tiles all split
+// (fewer than one wave of pairs) takes the paired kernel whenever there is a
+// workspace.
+static Tiled tiled_choice(int kind, int64_t m, int64_t n, int64_t k, bool ws, int64_t sms) {
+  const Tiled tk = tiled_kind(kind, m, n, sms);
+  if (ws) {
+    const PairPlan plan = pair_plan(m, n, k, std::max<int64_t>(1, sms / 2));
+    if (plan.split > 1 && plan.dp_tiles == 0) return Tiled::kPair;
+  }
+  return tk;
 }
 
 // Paired-SM kernel.  c8 != nullptr (mode 1 only): E4M3 output c8 =
-// E4M3(C / *s_out) instead of bf16 c.  split > 1: K split into that many parts
-// per tile, partials and counters in the workspace (pair_split_bytes(m, n,
-// split) bytes, counters zero).
+// E4M3(C / *s_out) instead of bf16 c.  workspace != nullptr
+// (pair_split_bytes(m, k, sms) bytes, counters zero): K split as pair_plan
+// says, partials and counters there.
 static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uint8_t* sfa, const uint8_t* sfb,
                                 int64_t m, int64_t n, int64_t k, const float* sa, const float* sb, void* c,
                                 int64_t ldc, cudaStream_t stream, const DeviceInfo& dev, uint8_t* c8 = nullptr,
-                                const float* s_out = nullptr, int split = 1, void* workspace = nullptr) {
+                                const float* s_out = nullptr, void* workspace = nullptr) {
   CUtensorMap ta, tb, tsa, tsb;
   fp8mm_status st = make_map(&ta, a, k, m, 128);
   if (st != FP8MM_OK) return st;
@@ -403,11 +427,8 @@ static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uin
   p.c8 = c8;
   p.s_out = s_out;
   p.group_m = pair_group_m(n, k);
-  p.split = split > 1 ? split : 1;
-  if (p.split > 1) {
-    p.partials = static_cast<float*>(workspace);
-    p.tickets = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + pair_partials_bytes(m, n, p.split));
-  }
+  p.split = 1;
+  p.dp_tiles = p.num_tiles;
   const void* kern = mx ? reinterpret_cast<const void*>(gemm_pair_kernel<true, 6, 1>)
                      : c8 ? reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2, true>)
                           : reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2>);
@@ -416,7 +437,16 @@ static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uin
   if ((st = ensure_smem(kern, smem, dev.device)) != FP8MM_OK) return st;
   int pairs = 0;
   if ((st = max_pairs(kern, smem, threads, dev, &pairs)) != FP8MM_OK) return st;
-  pairs = std::min(pairs, p.num_tiles * p.split);
+  if (workspace != nullptr) {
+    const PairPlan plan = pair_plan(m, n, k, std::min<int64_t>(pairs, std::max(1, dev.sms / 2)));
+    if (plan.split > 1) {
+      p.split = plan.split;
+      p.dp_tiles = plan.dp_tiles;
+      p.partials = static_cast<float*>(workspace);
+      p.tickets = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + pair_partials_bytes(dev.sms));
+    }
+  }
+  pairs = std::min(pairs, p.dp_tiles + (p.num_tiles - p.dp_tiles) * p.split);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -674,6 +704,16 @@ fp8mm_status fp8mm_sf_from_canonical(const uint8_t* canonical, int64_t rows, int
   return FP8MM_OK;
 }
 
+int32_t fp8mm_pair_split_plan(int64_t m, int64_t n, int64_t k, int32_t pairs, int32_t* dp_tiles) {
+  if (m <= 0 || n <= 0 || k <= 0 || pairs <= 0) {
+    if (dp_tiles != nullptr) *dp_tiles = 0;
+    return 1;
+  }
+  const PairPlan plan = pair_plan(m, n, k, pairs);
+  if (dp_tiles != nullptr) *dp_tiles = plan.dp_tiles;
+  return plan.split;
+}
+
 size_t fp8mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas) {
   if (m <= 0 || n <= 0 || k <= 0) return 0;
   int dev = 0, sms = 0;
@@ -681,7 +721,7 @@ size_t fp8mm_workspace_bytes(int64_t m, int64_t n, int64_t k, int32_t ctas) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0))
     sms = 148;
   cudaGetLastError();  // a host without a GPU leaves an error behind
-  if (m > 64) return pair_split_bytes(m, n, pair_split(m, n, k, sms));
+  if (m > 64) return pair_split_bytes(m, k, sms);
   int g = ctas > 0 ? ctas : sms;
   const int64_t units = cdiv(n, 128) * cdiv(k, 128);
   g = small_m_ctas(units, cdiv(n, 128), cdiv(k, 128), small_m_tile(m), ctas, g);
@@ -868,12 +908,10 @@ fp8mm_status fp8_gemm(const void* a_e4m3, const void* b_e4m3, int64_t m, int64_t
   const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
   const int split = tiled_split(opt, kind, m, n, k, dev.sms);
   if (split < 0) return FP8MM_ERR_WORKSPACE;
-  if (split > 1)
-    return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev,
-                       nullptr, nullptr, split, opt->workspace);
-  const Tiled tk = tiled_kind(kind, m, n, dev.sms);
+  const Tiled tk = tiled_choice(kind, m, n, k, split > 0, dev.sms);
   if (tk == Tiled::kPair)
-    return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev);
+    return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev,
+                       nullptr, nullptr, split > 0 ? opt->workspace : nullptr);
   return launch_tiled(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, c_bf16, ldc, s, dev,
                       nullptr, nullptr, tk == Tiled::k1SmN128);
 }
@@ -900,13 +938,10 @@ fp8mm_status fp8_gemm_e4m3_out(const void* a_e4m3, const void* b_e4m3, int64_t m
   const int kind = opt ? opt->kernel : FP8MM_KERNEL_AUTO;
   const int split = tiled_split(opt, kind, m, n, k, dev.sms);
   if (split < 0) return FP8MM_ERR_WORKSPACE;
-  if (split > 1)
-    return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, nullptr, ldc, s, dev, c8,
-                       scale_out, split, opt->workspace);
-  const Tiled tk = tiled_kind(kind, m, n, dev.sms);
+  const Tiled tk = tiled_choice(kind, m, n, k, split > 0, dev.sms);
   if (tk == Tiled::kPair)
     return launch_pair(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, nullptr, ldc, s, dev, c8,
-                       scale_out);
+                       scale_out, split > 0 ? opt->workspace : nullptr);
   return launch_tiled(false, a_e4m3, b_e4m3, nullptr, nullptr, m, n, k, scale_a, scale_b, nullptr, ldc, s, dev, c8,
                       scale_out, tk == Tiled::k1SmN128);
 }
@@ -932,11 +967,10 @@ fp8mm_status mxfp8_gemm(const void* a_e4m3, const uint8_t* sf_a, const void* b_e
   if (small) return launch_small_m(a_e4m3, sf_a, b_e4m3, sf_b, m, n, k, c_bf16, ldc, opt, s, dev);
   const int split = tiled_split(opt, kind, m, n, k, dev.sms);
   if (split < 0) return FP8MM_ERR_WORKSPACE;
-  if (split > 1)
+  const Tiled tk = tiled_choice(kind, m, n, k, split > 0, dev.sms);
+  if (tk == Tiled::kPair)
     return launch_pair(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev, nullptr,
-                       nullptr, split, opt->workspace);
-  const Tiled tk = tiled_kind(kind, m, n, dev.sms);
-  if (tk == Tiled::kPair) return launch_pair(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev);
+                       nullptr, split > 0 ? opt->workspace : nullptr);
   return launch_tiled(true, a_e4m3, b_e4m3, sf_a, sf_b, m, n, k, nullptr, nullptr, c_bf16, ldc, s, dev, nullptr,
                       nullptr, tk == Tiled::k1SmN128);
 }

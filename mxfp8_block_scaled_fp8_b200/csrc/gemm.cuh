@@ -15,8 +15,9 @@
 // 256-wide tiles would leave most SMs idle.  Warp roles:
 //   warp 0      TMA producer: A/B tiles (128-byte swizzle) and, in mode 2,
 //               the 512-byte scale chunks, into a kStages-deep ring.
-//   warp 1      allocates TMEM; one lane issues tcgen05.mma (and tcgen05.cp of
-//               the scale chunks) per 128-byte K slab, commits to free the slab.
+//   warp 1      allocates TMEM; one elected lane of the converged warp issues
+//               tcgen05.mma (and tcgen05.cp of the scale chunks) per 128-byte K
+//               slab, commits to free the slab.
 //   warps 2..9  epilogue: each drains half a tile row-block of the fp32
 //               accumulator into registers (tcgen05.ld, one wait), frees the
 //               accumulator, then scales, converts to bf16 RNE and stores
@@ -54,9 +55,10 @@ struct GemmArgs {
   int sfb_row_tiles;         // ceil(n / 128): 128-row tiles present in sfb
   uint64_t timeout_ns;
   int group_m;               // paired-SM kernel: 256-row tiles per raster group
-  int split;                 // paired-SM kernel: K parts per tile (1 = whole K, no partials)
-  float* partials;           // split > 1: fp32 partials [num_tiles * split][2][128 * 256]
-  unsigned* tickets;         // split > 1: arrivals per (tile, CTA rank), zero between calls
+  int split;                 // paired-SM kernel: K parts per split tile (1 = whole K, no partials)
+  int dp_tiles;              // paired-SM kernel: tiles [0, dp_tiles) run whole, the rest in split parts
+  float* partials;           // split > 1: fp32 partials [(num_tiles - dp_tiles) * split][2][128 * 256]
+  unsigned* tickets;         // split > 1: arrivals per (split tile, CTA rank), zero between calls
 };
 
 // Per-token / per-channel scaling of an fp32 accumulator, sa * sb * acc
@@ -214,7 +216,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues (see elect_one_sync).
+    {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
@@ -225,23 +228,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int sfb_chunks = 0;
         if constexpr (kMX) sfb_chunks = min(Cfg::kSfbChunks, p.sfb_row_tiles - nb * Cfg::kSfbChunks);
         for (int kb = 0; kb < p.num_k; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) {
+          if (!warp_wait(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) {
             ok = false;
             break;
           }
-          uint32_t bytes = Cfg::kABytes + Cfg::kBBytes;
-          if constexpr (kMX) bytes += 512u + 512u * sfb_chunks;
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(smem + Cfg::kOffA + stage * Cfg::kABytes, &tmA, &full[stage], kb * kBK, mb * kBM);
-          tma_load_2d(smem + Cfg::kOffB + stage * Cfg::kBBytes, &tmB, &full[stage], kb * kBK, nb * kBN);
-          if constexpr (kMX) {
-            bulk_load(smem + Cfg::kOffSfa + stage * 512, p.sfa + (static_cast<int64_t>(mb) * p.n_kc + kb) * 512,
-                      512u, &full[stage]);
-            for (int i = 0; i < sfb_chunks; ++i)
-              bulk_load(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes + i * 512,
-                        p.sfb + (static_cast<int64_t>(nb * Cfg::kSfbChunks + i) * p.n_kc + kb) * 512, 512u,
-                        &full[stage]);
+          if (elect_one_sync()) {
+            uint32_t bytes = Cfg::kABytes + Cfg::kBBytes;
+            if constexpr (kMX) bytes += 512u + 512u * sfb_chunks;
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            tma_load_2d(smem + Cfg::kOffA + stage * Cfg::kABytes, &tmA, &full[stage], kb * kBK, mb * kBM);
+            tma_load_2d(smem + Cfg::kOffB + stage * Cfg::kBBytes, &tmB, &full[stage], kb * kBK, nb * kBN);
+            if constexpr (kMX) {
+              bulk_load(smem + Cfg::kOffSfa + stage * 512, p.sfa + (static_cast<int64_t>(mb) * p.n_kc + kb) * 512,
+                        512u, &full[stage]);
+              for (int i = 0; i < sfb_chunks; ++i)
+                bulk_load(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes + i * 512,
+                          p.sfb + (static_cast<int64_t>(nb * Cfg::kSfbChunks + i) * p.n_kc + kb) * 512, 512u,
+                          &full[stage]);
+            }
           }
+          __syncwarp();
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -250,7 +256,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      // Let every copy this thread started land before the CTA can exit.
+      // Let every copy the warp started land before the CTA can exit.
       for (int s = 0; s < kStages; ++s)
         if (issued_mask & (1u << s))
           mbar_wait(&full[s], (issued_parity >> s) & 1u, p.timeout_ns, nullptr, kSiteProducerDrain);
@@ -258,56 +264,62 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues (see elect_one_sync).
+    {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
-        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, kSiteMmaAccEmpty)) break;
+        if (!warp_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, kSiteMmaAccEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
         for (int kb = 0; kb < p.num_k; ++kb) {
-          if (!mbar_wait(&full[stage], phase, p.timeout_ns, abort_flag, kSiteMmaFull)) {
+          if (!warp_wait(&full[stage], phase, p.timeout_ns, abort_flag, kSiteMmaFull)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t adesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffA + stage * Cfg::kABytes));
-          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffB + stage * Cfg::kBBytes));
-          if constexpr (kMX) {
-            const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(Cfg::kSfCol0 + stage * Cfg::kSfColsPerStage);
-            const uint32_t sfb_t = sfa_t + 4u;
-            tmem_cp_32x128b_warpx4(sfa_t, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfa + stage * 512)));
+          if (elect_one_sync()) {
+            const uint64_t adesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffA + stage * Cfg::kABytes));
+            const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffB + stage * Cfg::kBBytes));
+            if constexpr (kMX) {
+              const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(Cfg::kSfCol0 + stage * Cfg::kSfColsPerStage);
+              const uint32_t sfb_t = sfa_t + 4u;
+              tmem_cp_32x128b_warpx4(sfa_t, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfa + stage * 512)));
 #pragma unroll
-            for (int i = 0; i < Cfg::kSfbChunks; ++i)
-              tmem_cp_32x128b_warpx4(sfb_t + 4u * i,
-                                     sf_chunk_desc(smem_u32(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes + i * 512)));
+              for (int i = 0; i < Cfg::kSfbChunks; ++i)
+                tmem_cp_32x128b_warpx4(
+                    sfb_t + 4u * i, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes + i * 512)));
 #pragma unroll
-            for (int kk = 0; kk < kBK / kMmaK; ++kk)
-              mma_mxf8f6f4(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8f6f4(kBM, kBN, kk, kk), sfa_t, sfb_t,
-                           (kb | kk) != 0);
-          } else {
+              for (int kk = 0; kk < kBK / kMmaK; ++kk)
+                mma_mxf8f6f4(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8f6f4(kBM, kBN, kk, kk), sfa_t,
+                             sfb_t, (kb | kk) != 0);
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < kBK / kMmaK; ++kk)
-              mma_f8f6f4(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_f8f6f4(kBM, kBN), (kb | kk) != 0);
+              for (int kk = 0; kk < kBK / kMmaK; ++kk)
+                mma_f8f6f4(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_f8f6f4(kBM, kBN), (kb | kk) != 0);
+            }
+            tc_commit(&empty[stage]);
           }
-          tc_commit(&empty[stage]);
+          __syncwarp();
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(&acc_full[acc]);
+        if (elect_one_sync()) tc_commit(&acc_full[acc]);
+        __syncwarp();
         if (++acc == kAccStages) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
-      // Every MMA / copy this thread issued must finish before TMEM is freed.
-      tc_commit(drain);
+      // Every MMA / copy the warp issued must finish before TMEM is freed.
+      if (elect_one_sync()) tc_commit(drain);
+      __syncwarp();
       mbar_wait(drain, 0, p.timeout_ns, nullptr, kSiteDrain);
     }
     __syncwarp();

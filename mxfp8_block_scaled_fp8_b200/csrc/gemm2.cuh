@@ -25,14 +25,18 @@
 // release arrivals from those warps made the kernel ~45 % slower.
 //
 // Warp roles per CTA: warp 0 TMA producer; warp 1 TMEM owner and, on rank 0,
-// MMA issuer; warps 2..17 epilogue (four per TMEM sub-partition, 64
-// accumulator columns each, drained into registers with one wait so the
-// accumulator is free again at once).
+// MMA issuer (the whole warp, one elected lane issuing); warps 2..17
+// epilogue (four per TMEM sub-partition, 64 accumulator columns each,
+// drained into registers with one wait so the accumulator is free again at
+// once).
 //
-// Split K (split > 1, for shapes whose tiles fill less than one wave of SM
-// pairs): the work units are (tile, K part) with part j covering K slabs
-// [floor(j*num_k/split), floor((j+1)*num_k/split)); pairs take units in turn.
-// Each CTA stores its fp32 partial (its 128 rows x 256 columns) in the
+// Split K (split > 1): tiles [0, dp_tiles) are whole work units; each later
+// tile is `split` units (tile, K part), part j covering K slabs
+// [floor(j*num_k/split), floor((j+1)*num_k/split)).  Pairs take units in
+// turn, so with dp_tiles a multiple of the pair count the split tiles form
+// the last round: where the tiles fill less than one wave all are split
+// (dp_tiles = 0), else only those of the last, partly filled wave.  Each CTA
+// of a split unit stores its fp32 partial (its 128 rows x 256 columns) in the
 // workspace, bumps the (tile, rank) arrival counter, and the last to arrive
 // sums the parts in part order (fixed, so the result does not depend on
 // timing), applies the scales, writes C and resets the counter.  No CTA waits
@@ -89,8 +93,16 @@ __device__ __forceinline__ void pair_tile_coords(int t, const GemmArgs& p, int& 
 
 // Work unit u: tile t and its K slabs [kb0, kb1).
 __device__ __forceinline__ void pair_unit(int u, const GemmArgs& p, int& t, int& kb0, int& kb1) {
-  t = u / p.split;
-  const int j = u - t * p.split;
+  if (u < p.dp_tiles) {
+    t = u;
+    kb0 = 0;
+    kb1 = p.num_k;
+    return;
+  }
+  const int v = u - p.dp_tiles;
+  const int q = v / p.split;
+  t = p.dp_tiles + q;
+  const int j = v - q * p.split;
   kb0 = static_cast<int>(static_cast<int64_t>(j) * p.num_k / p.split);
   kb1 = static_cast<int>(static_cast<int64_t>(j + 1) * p.num_k / p.split);
 }
@@ -121,7 +133,7 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 4);
   volatile int* last_flag = reinterpret_cast<volatile int*>(smem + Cfg::kOffMisc + 8);
-  const int num_units = p.num_tiles * p.split;
+  const int num_units = p.dp_tiles + (p.num_tiles - p.dp_tiles) * p.split;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -163,7 +175,8 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues (see elect_one_sync).
+    {
       int stage = 0;
       uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
       bool ok = true;
@@ -172,19 +185,22 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
         pair_unit(u, p, t, kb0, kb1);
         pair_tile_coords(t, p, mb, nb);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) {
+          if (!warp_wait_cluster(&empty[stage], phase ^ 1u, p.timeout_ns, abort_flag, kSiteProducerEmpty)) {
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(&full[stage], Cfg::kTxPair);
-          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
-          tma_load_2d_pair(smem + Cfg::kOffA + stage * Cfg::kABytes, &tmA, fb, kb * kBK, mb * 256 + rank * 128);
-          tma_load_2d_pair(smem + Cfg::kOffB + stage * Cfg::kBBytes, &tmB, fb, kb * kBK, nb * 256 + rank * 128);
-          if constexpr (kMX) {
-            tma_load_3d_pair(smem + Cfg::kOffSfa + stage * Cfg::kSfaBytes, &tmSFA, fb, 0, kb, mb * 2 + rank);
-            // both B chunks, four replicas each, in one load (a zero-stride replica dimension)
-            tma_load_4d_pair(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes, &tmSFB, fb, 0, kb, 0, nb * 2);
+          if (elect_one_sync()) {
+            if (leader) mbar_arrive_expect_tx(&full[stage], Cfg::kTxPair);
+            const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+            tma_load_2d_pair(smem + Cfg::kOffA + stage * Cfg::kABytes, &tmA, fb, kb * kBK, mb * 256 + rank * 128);
+            tma_load_2d_pair(smem + Cfg::kOffB + stage * Cfg::kBBytes, &tmB, fb, kb * kBK, nb * 256 + rank * 128);
+            if constexpr (kMX) {
+              tma_load_3d_pair(smem + Cfg::kOffSfa + stage * Cfg::kSfaBytes, &tmSFA, fb, 0, kb, mb * 2 + rank);
+              // both B chunks, four replicas each, in one load (a zero-stride replica dimension)
+              tma_load_4d_pair(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes, &tmSFB, fb, 0, kb, 0, nb * 2);
+            }
           }
+          __syncwarp();
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) {
@@ -210,52 +226,60 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer (rank 0 only)
-    if (leader && lane == 0) {
+    // The whole warp runs the loop; one elected lane issues (see elect_one_sync).
+    if (leader) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int u = pair; ok && u < num_units; u += npairs) {
         int t, kb0, kb1;
         pair_unit(u, p, t, kb0, kb1);
-        if (!mbar_wait_cluster(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, kSiteMmaAccEmpty)) break;
+        if (!warp_wait_cluster(&acc_empty[acc], acc_phase ^ 1u, p.timeout_ns, abort_flag, kSiteMmaAccEmpty)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait_cluster(&full[stage], phase, p.timeout_ns, abort_flag, kSiteMmaFull)) {
+          if (!warp_wait_cluster(&full[stage], phase, p.timeout_ns, abort_flag, kSiteMmaFull)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t adesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffA + stage * Cfg::kABytes));
-          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffB + stage * Cfg::kBBytes));
-          if constexpr (kMX) {
-            const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(Cfg::kSfCol0 + stage * Cfg::kSfColsPerStage);
-            tmem_cp_32x128b_warpx4_pair(sfa_t, sf_chunk_desc(smem_u32(smem + Cfg::kOffSfa + stage * Cfg::kSfaBytes)));
-            tmem_cp_128x256b_pair(sfa_t + 8u,
-                                  sf_replicated_desc(smem_u32(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes), 2048u));
+          if (elect_one_sync()) {
+            const uint64_t adesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffA + stage * Cfg::kABytes));
+            const uint64_t bdesc = sw128_kmajor_desc(smem_u32(smem + Cfg::kOffB + stage * Cfg::kBBytes));
+            if constexpr (kMX) {
+              const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(Cfg::kSfCol0 + stage * Cfg::kSfColsPerStage);
+              tmem_cp_32x128b_warpx4_pair(sfa_t,
+                                          sf_chunk_desc(smem_u32(smem + Cfg::kOffSfa + stage * Cfg::kSfaBytes)));
+              tmem_cp_128x256b_pair(sfa_t + 8u,
+                                    sf_replicated_desc(smem_u32(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes), 2048u));
 #pragma unroll
-            for (int kk = 0; kk < kBK / kMmaK; ++kk)
-              mma_mxf8f6f4_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8f6f4(256, 256, kk, kk), sfa_t,
-                                sfa_t + 8u, kb != kb0 || kk != 0);
-          } else {
+              for (int kk = 0; kk < kBK / kMmaK; ++kk)
+                mma_mxf8f6f4_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8f6f4(256, 256, kk, kk), sfa_t,
+                                  sfa_t + 8u, kb != kb0 || kk != 0);
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < kBK / kMmaK; ++kk)
-              mma_f8f6f4_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_f8f6f4(256, 256), kb != kb0 || kk != 0);
+              for (int kk = 0; kk < kBK / kMmaK; ++kk)
+                mma_f8f6f4_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_f8f6f4(256, 256),
+                                kb != kb0 || kk != 0);
+            }
+            tc_commit_pair_mc(&empty[stage], 0x3);
           }
-          tc_commit_pair_mc(&empty[stage], 0x3);
+          __syncwarp();
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit_pair_mc(&acc_full[acc], 0x3);
+        if (elect_one_sync()) tc_commit_pair_mc(&acc_full[acc], 0x3);
+        __syncwarp();
         if (++acc == kAccStages) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
-      tc_commit_pair_mc(drain, 0x1);
+      if (elect_one_sync()) tc_commit_pair_mc(drain, 0x1);
+      __syncwarp();
       mbar_wait(drain, 0, p.timeout_ns, nullptr, kSiteDrain);
     }
     __syncwarp();
@@ -306,9 +330,10 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
       const int row = mb * 256 + static_cast<int>(rank) * 128 + sp * 32 + lane;
       float s_row = 1.f;
       if constexpr (!kMX) s_row = (row < p.m) ? __ldg(p.sa + row) : 0.f;
-      if (p.split > 1) {
+      if (u >= p.dp_tiles) {
         // Publish this part, count it; the last part to arrive reduces.
-        float* mine = p.partials + (static_cast<int64_t>(u) * 2 + rank) * kPairPartFloats + wl * 2048 + lane;
+        float* mine =
+            p.partials + (static_cast<int64_t>(u - p.dp_tiles) * 2 + rank) * kPairPartFloats + wl * 2048 + lane;
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
@@ -319,7 +344,7 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
         // last part's increment acquires every earlier part's stores, and the
         // barrier after it hands them to its other threads.
         if (!epi_meet()) break;
-        unsigned* ticket = p.tickets + static_cast<int64_t>(t) * 2 + rank;
+        unsigned* ticket = p.tickets + static_cast<int64_t>(t - p.dp_tiles) * 2 + rank;
         if (threadIdx.x == Cfg::kEpiWarp0 * 32) {
           unsigned prev;
           asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ticket) : "memory");
@@ -334,8 +359,9 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = 0.f;
           for (int part = 0; part < p.split; ++part) {
-            const float* src = p.partials + (static_cast<int64_t>(t * p.split + part) * 2 + rank) * kPairPartFloats +
-                               wl * 2048 + ch * 1024 + lane;
+            const float* src =
+                p.partials + (static_cast<int64_t>((t - p.dp_tiles) * p.split + part) * 2 + rank) * kPairPartFloats +
+                wl * 2048 + ch * 1024 + lane;
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] += __ldcg(src + j * 32);
           }

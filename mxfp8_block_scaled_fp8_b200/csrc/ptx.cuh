@@ -269,6 +269,35 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   if (mbar_try_wait_cluster(bar, parity)) return true;
   return mbar_wait_cluster_slow(bar, parity, timeout_ns, abort, site);
 }
+
+// ------------------------------------------------------------ warp-converged issue
+// The tcgen05 MMA and copy instructions are issued by one thread, but issued
+// from a lane of a warp whose other lanes have diverged away they are slow:
+// measured on B200 in the paired MX GEMM (8192 x 22016 x 8192), issuing the
+// scale copies and MMAs from lane 0 alone took 1196 us, from one lane chosen
+// by elect.sync in a converged warp 1081 us (the copies' cost fell from 212
+// to 63 us with the loads removed).  So the issuing warps run their loops
+// with every lane, wait together, and let one elected lane issue.
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+// Bounded waits by every lane of the calling warp, which continues, converged,
+// only if all lanes saw the phase complete (a wait that expired or saw
+// *abort gives false in every lane).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, volatile int* abort,
+                                          unsigned site) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, timeout_ns, abort, site));
+}
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
+                                                  volatile int* abort, unsigned site) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait_cluster(bar, parity, timeout_ns, abort, site));
+}
 // Tiled TMA load into this CTA's shared memory whose completion bytes go to
 // the mbarrier at `mbar_cluster_addr`, which may be in the peer CTA of the
 // pair (cta_group::2).  Not a multicast load.

@@ -66,6 +66,7 @@ _SIGNATURES = {
     "fp8mm_sf_to_canonical": ([_P, _I64, _I64, _P], ctypes.c_int),
     "fp8mm_sf_from_canonical": ([_P, _I64, _I64, _P], ctypes.c_int),
     "fp8mm_workspace_bytes": ([_I64, _I64, _I64, ctypes.c_int32], ctypes.c_size_t),
+    "fp8mm_pair_split_plan": ([_I64, _I64, _I64, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int32),
     "fp8mm_quantize_gemm_workspace_bytes": ([_I64, _I64, _I64, ctypes.c_int32], ctypes.c_size_t),
     "fp8mm_status_str": ([ctypes.c_int], ctypes.c_char_p),
     "fp8mm_last_cuda_error": ([], ctypes.c_int),
@@ -142,8 +143,8 @@ def fp8_gemm(a: torch.Tensor, b: torch.Tensor, scale_a: torch.Tensor, scale_b: t
              c: torch.Tensor | None = None, kernel: int = KERNEL_AUTO, stream=None,
              workspace: torch.Tensor | None = None) -> torch.Tensor:
     """C bf16 [m, n] = diag(scale_a) (A x B^T) diag(scale_b); a [m,k], b [n,k] E4M3 codes.
-    workspace (zeroed once, workspace_bytes(m, n, k) bytes): lets m > 64 shapes that fill less than one
-    wave of SM pairs split K over the pairs."""
+    workspace (zeroed once, workspace_bytes(m, n, k) bytes): lets m > 64 shapes split the K range of the
+    tiles of their last, partly filled wave of SM pairs over the pairs."""
     a, b = _u8(a), _u8(b)
     _need(a, torch.uint8, "a"); _need(b, torch.uint8, "b")
     _need(scale_a, torch.float32, "scale_a"); _need(scale_b, torch.float32, "scale_b")
@@ -275,6 +276,13 @@ def workspace_bytes(m: int, n: int, k: int, ctas: int = 0) -> int:
     return int(lib().fp8mm_workspace_bytes(m, n, k, ctas))
 
 
+def pair_split_plan(m: int, n: int, k: int, pairs: int) -> tuple[int, int]:
+    """(K parts per split tile, tiles run whole) of the paired kernel's split with `pairs` SM pairs."""
+    dp = ctypes.c_int32(0)
+    split = int(lib().fp8mm_pair_split_plan(m, n, k, pairs, ctypes.byref(dp)))
+    return split, int(dp.value)
+
+
 def quantize_gemm_workspace_bytes(m: int, n: int, k: int, ctas: int = 0) -> int:
     return int(lib().fp8mm_quantize_gemm_workspace_bytes(m, n, k, ctas))
 
@@ -286,7 +294,7 @@ def mxfp8_gemm(a: torch.Tensor, sf_a: torch.Tensor, b: torch.Tensor, sf_b: torch
     """C bf16 [m, n] = block-scaled A x B^T; a [m,k], b [n,k] codes with their library-layout scales.
     workspace (zeroed once, workspace_bytes(m, n, k, small_m_ctas) bytes): the small-M kernel's stream-K
     split for m <= 64 where the CTA count is not tile-aligned (aligned splits reduce inside clusters);
-    for m > 64 the K split of shapes that fill less than one wave of SM pairs.
+    for m > 64 the K split of the tiles of the last, partly filled wave of SM pairs.
     weights_ready: b and sf_b were complete before the preceding kernel on the stream started (see
     FP8MM_FLAG_WEIGHTS_READY).  split_via_workspace: FP8MM_FLAG_SPLIT_VIA_WORKSPACE.  sf_a_8x4: sf_a is in
     the small-M layout of mxfp8_quantize_8x4 (m <= 64 only)."""

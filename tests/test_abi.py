@@ -103,17 +103,15 @@ def test_workspace_sizes():
     # 2 * G * 128 * NM floats (256-byte aligned) + one counter per 128-row tile
     assert fp8mm.workspace_bytes(64, 14336, 4096, 148) == 2 * 148 * 128 * 64 * 4 + 512
     assert fp8mm.workspace_bytes(1, 4096, 14336, 148) == 2 * 148 * 128 * 16 * 4 + 256
-    # m > 64: the paired kernel's K split, on a host without a GPU for 148 SMs (74 pairs);
-    # partials of 128 x 256 fp32 per (tile, part, CTA rank), then 2 counters per tile (256-byte rounded)
+    # m > 64 and K >= 8192 (64 slabs of 128): the paired kernel's K split, on a host without a GPU for
+    # 148 SMs (74 pairs), whatever the tile count: room for one split part per pair, 128 x 256 fp32 per CTA
+    # rank, then 2 counters per pair (256-byte rounded); shorter K is never split
     part = 128 * 256 * 4
-    assert fp8mm.workspace_bytes(65, 4096, 8192, 148) == 16 * 4 * 2 * part + 256     # 16 tiles, 4 parts
-    assert fp8mm.workspace_bytes(512, 2048, 8192) == 16 * 4 * 2 * part + 256         # the same tiles
-    assert fp8mm.workspace_bytes(2048, 512, 16384) == 16 * 4 * 2 * part + 256        # 128 slabs: 74 // 16 = 4
-    assert fp8mm.workspace_bytes(1024, 1024, 8192) == 16 * 4 * 2 * part + 256
-    assert fp8mm.workspace_bytes(2048, 1024, 8192) == 32 * 2 * 2 * part + 256        # 32 tiles, 2 parts
-    assert fp8mm.workspace_bytes(2048, 1024, 4096) == 0                              # 32 K slabs: no split
+    for shape in [(65, 4096, 8192), (512, 2048, 8192), (2048, 512, 16384), (2048, 1024, 8192),
+                  (8192, 22016, 8192), (8192, 2048, 8192)]:
+        assert fp8mm.workspace_bytes(*shape) == 74 * 2 * part + 768, shape
+    assert fp8mm.workspace_bytes(2048, 1024, 4096) == 0                              # 32 K slabs
     assert fp8mm.workspace_bytes(65, 4096, 4096) == 0
-    assert fp8mm.workspace_bytes(8192, 22016, 8192) == 0                             # more tiles than pairs
     assert fp8mm.workspace_bytes(8, 128, 128, 148) == 2 * 1 * 128 * 16 * 4 + 256   # clamped to 1 unit
     # the small-M kernel's automatic CTA count (a host without a GPU counts 148 SMs), read back from the
     # partials' size: tile-aligned counts (s CTAs per 128-row weight tile, s dividing its K slabs) where one
@@ -193,3 +191,27 @@ def test_sf8x4_argument_errors_without_gpu():
     assert L.mxfp8_quantize_8x4(None, 4, 48, 48, None, 48, None, None) == 2      # k % 32
     assert L.mxfp8_quantize_8x4(None, 4, 64, 64, None, 64, None, None) == 1      # null pointers
     assert L.mxfp8_quantize_8x4(None, 0, 64, 64, None, 64, None, None) == 0      # nothing to do
+
+
+def test_pair_split_plan():
+    """The paired kernel's split plan: (K parts per split tile, tiles run whole).  The tiles of the last,
+    partly filled wave of pairs are split into as many parts as fit the pairs it leaves (all tiles where
+    they fill less than one wave), each of >= 16 K slabs of 128, <= 8 parts; none for m <= 64, K < 8192
+    or whole waves."""
+    plan = fp8mm.pair_split_plan
+    assert plan(8192, 22016, 8192, 74) == (4, 2738)      # 2752 tiles: 37 waves + 14; 74 // 14 = 5 > 64 // 16
+    assert plan(8192, 2048, 8192, 74) == (2, 222)        # 256 tiles: 3 waves + 34
+    assert plan(2560, 2048, 8192, 74) == (4, 74)         # 80 tiles: 1 wave + 6
+    assert plan(8192, 3584, 8192, 74) == (4, 444)        # 448 tiles: 6 waves + 4
+    assert plan(8192, 9472, 8192, 74) == (1, 1184)       # 16 whole waves
+    assert plan(8192, 3840, 8192, 74) == (2, 444)        # 480 tiles: 6 waves + 36; 74 // 36 = 2
+    assert plan(8192, 4096, 8192, 74) == (1, 512)        # 512 tiles: 6 waves + 68; no room for 2 parts
+    assert plan(512, 2048, 8192, 74) == (4, 0)           # 16 tiles, all split
+    assert plan(2048, 1024, 8192, 74) == (2, 0)
+    assert plan(300, 600, 8960, 74) == (4, 0)            # 70 slabs
+    assert plan(2048, 512, 32768, 74) == (4, 0)          # 16 tiles: 74 // 16 = 4 parts of 64 slabs
+    assert plan(512, 256, 32768, 74) == (8, 0)           # 2 tiles: capped at 8 parts
+    assert plan(2048, 1024, 4096, 74) == (1, 32)         # 32 K slabs: never split
+    assert plan(64, 4096, 8192, 74) == (1, 16)           # m <= 64: the small-M kernel's business
+    assert plan(8192, 22016, 8192, 72) == (4, 2736)      # 72 pairs: 38 waves + 16; 72 // 16 = 4
+    assert plan(0, 128, 128, 74) == (1, 0)

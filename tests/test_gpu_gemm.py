@@ -330,6 +330,71 @@ def test_edge_values_tiled(mode, kernel):
 
 
 def test_attn_rowwise_full():
-    """The attention-shaped per-token GEMM 8192 x 2048 x 8192 in full."""
+    """The attention-shaped per-token GEMM 8192 x 2048 x 8192 in full, without and with a workspace (256
+    tiles: with 74 SM pairs the 34 tiles of the last wave run as 2 K parts each)."""
+    import oracle as orc
     a, bt = synthetic.attn()
-    run_rowwise(a, bt, label="attn 8192x2048x8192 full")
+    m, n, k = a.shape[0], bt.shape[0], a.shape[1]
+    qa, sa = orc.quantize_rowwise(synthetic.bits(a))
+    qb, sb = orc.quantize_rowwise(synthetic.bits(bt))
+    ga, gsa = fp8mm.fp8_quantize_rowwise(gu.to_dev(a))
+    gb, gsb = fp8mm.fp8_quantize_rowwise(gu.to_dev(bt))
+    ws = _ws(m, n, k)
+    c_plain = fp8mm.fp8_gemm(ga, gb, gsa, gsb)
+    c_split = fp8mm.fp8_gemm(ga, gb, gsa, gsb, workspace=ws)
+    torch.cuda.synchronize()
+    c_ref, bound = orc.gemm_rowwise(qa, qb, sa, sb)
+    gu.check_gemm(c_plain, c_ref, bound, "attn 8192x2048x8192 full")
+    gu.check_gemm(c_split, c_ref, bound, "attn 8192x2048x8192 full, last wave split")
+    assert not ws[-256:].any()
+    assert fp8mm.last_device_error() == 0
+
+
+def _tiles_equal(c1, c2):
+    """Per 256 x 256 output tile: whether the two results are bit-identical there."""
+    m, n = c1.shape
+    return [[bool(torch.equal(c1[i:i + 256, j:j + 256], c2[i:i + 256, j:j + 256])) for j in range(0, n, 256)]
+            for i in range(0, m, 256)]
+
+
+@pytest.mark.parametrize("mode", ["mx", "rowwise"])
+def test_tail_split_full(mode):
+    """More tiles than SM pairs, with a workspace: the tiles of the last, partly filled wave split their K
+    range over the pairs (2560 x 2040 x 8192: 80 tiles, with 74 pairs the last 6 in raster order in 4 parts;
+    a ragged last column of tiles).  The full result meets the bar; a second call is bit-identical and
+    leaves the counters at zero; the tiles run whole equal a call without a workspace bit for bit, and no
+    more tiles than the last wave differ."""
+    import oracle as orc
+    m, n, k = 2560, 2040, 8192
+    a = synthetic.random_bf16((m, k), seed=71)
+    bt = synthetic.random_bf16((n, k), seed=72, sigma=0.05)
+    ws = _ws(m, n, k)
+    if mode == "mx":
+        qa, sfa = orc.mx_quantize(synthetic.bits(a))
+        qb, sfb = orc.mx_quantize(synthetic.bits(bt))
+        ga, gsfa = fp8mm.mxfp8_quantize(gu.to_dev(a))
+        gb, gsfb = fp8mm.mxfp8_quantize(gu.to_dev(bt))
+        call = lambda w: fp8mm.mxfp8_gemm(ga, gsfa, gb, gsfb, workspace=w)
+        ref = lambda: orc.gemm_mx(qa, sfa, qb, sfb)
+    else:
+        qa, sa = orc.quantize_rowwise(synthetic.bits(a))
+        qb, sb = orc.quantize_rowwise(synthetic.bits(bt))
+        ga, gsa = fp8mm.fp8_quantize_rowwise(gu.to_dev(a))
+        gb, gsb = fp8mm.fp8_quantize_rowwise(gu.to_dev(bt))
+        call = lambda w: fp8mm.fp8_gemm(ga, gb, gsa, gsb, workspace=w)
+        ref = lambda: orc.gemm_rowwise(qa, qb, sa, sb)
+    c_plain = call(None)
+    c1 = call(ws)
+    c2 = call(ws)
+    torch.cuda.synchronize()
+    assert torch.equal(c1, c2)
+    assert not ws[-256:].any()
+    assert fp8mm.last_device_error() == 0
+    same = _tiles_equal(c1, c_plain)
+    tiles = sum(len(r) for r in same)
+    differ = tiles - sum(sum(r) for r in same)
+    split, dp = fp8mm.pair_split_plan(m, n, k, 74)
+    assert (split, dp) == (4, 74)
+    assert differ <= tiles - dp, (differ, tiles - dp)
+    c_ref, bound = ref()
+    gu.check_gemm(c1, c_ref, bound, f"tail split {mode} {m}x{n}x{k}")
