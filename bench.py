@@ -413,11 +413,50 @@ def _sustained(step, gemm, stream, local, pci, seconds: float = 3.0, k: int = 10
             "note": "after several seconds of back-to-back steps (power cap); each call timed alone, median"}
 
 
-def _yardstick(torch, dev):
+def _best_of(torch, f, reps: int = 10):
+    for _ in range(3):
+        f()
+    torch.cuda.synchronize()
+    best = None
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        f()
+        e1.record()
+        e1.synchronize()
+        t = e0.elapsed_time(e1)
+        best = t if best is None else min(best, t)
+    return best
+
+
+def _yardstick(torch, dev, mx=None):
     """torch._scaled_mm (cuBLASLt FP8) on the same GPU in the same run: a
-    library yardstick, not a target and not the roofline denominator."""
+    library yardstick, not a target and not the roofline denominator.  mx =
+    (qx, sfx, qw, sfw, ours): the step's own MXFP8 operands, whose scale
+    layout is the one cuBLASLt reads for 1x32 UE8M0 block scales, timed
+    through cuBLASLt and through our call `ours` in the same protocol."""
     out = {"what": "torch._scaled_mm e4m3 x e4m3 -> bf16, best of 10 calls after 3 warm-up calls; "
                    "a library yardstick, not a target"}
+    if mx is not None:
+        try:
+            qx, sfx, qw, sfw, ours = mx
+            m, k = qx.shape
+            n = qw.shape[0]
+            a8, b8 = qx.view(torch.float8_e4m3fn), qw.view(torch.float8_e4m3fn)
+            sa, sb = sfx.view(torch.float8_e8m0fnu), sfw.view(torch.float8_e8m0fnu)
+            f = lambda: torch._scaled_mm(a8, b8.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
+            ref = f()
+            c = ours()
+            torch.cuda.synchronize()
+            diff = float((ref.float() - c.float()).abs().max())
+            tl, to = _best_of(torch, f), _best_of(torch, ours)
+            fl = 2.0 * m * n * k
+            out[f"{m}x{n}x{k}_mxfp8_cublaslt"] = {"ms": tl, "TFLOPS": fl / (tl * 1e-3) / 1e12,
+                                                  "max_abs_diff_vs_ours": diff}
+            out[f"{m}x{n}x{k}_mxfp8_ours_same_protocol"] = {"ms": to, "TFLOPS": fl / (to * 1e-3) / 1e12}
+            del ref, c
+        except Exception as e:  # a library limitation is reported, not fatal
+            out["mxfp8_error"] = f"{type(e).__name__}: {e}"[:200]
     try:
         shapes = {"8192x8192x8192_per_tensor": (8192, 8192, 8192, False),
                   "8192x22016x8192_rowwise": (8192, 22016, 8192, True),
@@ -428,18 +467,7 @@ def _yardstick(torch, dev):
             sa = torch.ones((m, 1) if rowwise else (), device=dev)
             sb = torch.ones((1, n) if rowwise else (), device=dev)
             f = lambda: torch._scaled_mm(a, b.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
-            for _ in range(3):
-                f()
-            torch.cuda.synchronize()
-            best = None
-            for _ in range(10):
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                f()
-                e1.record()
-                e1.synchronize()
-                t = e0.elapsed_time(e1)
-                best = t if best is None else min(best, t)
+            best = _best_of(torch, f)
             out[name] = {"ms": best, "TFLOPS": 2.0 * m * n * k / (best * 1e-3) / 1e12}
             del a, b
     except Exception as e:  # a library limitation is reported, not fatal
@@ -571,7 +599,9 @@ def run_ours(args):
     if not args.no_sustained:
         sustained = _sustained(step, lambda: fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c, workspace=gws), stream, local,
                                pci)
-    yard = _yardstick(torch, dev) if (rank == 0 and not args.no_rows) else None
+    yard = None
+    if rank == 0 and not args.no_rows:
+        yard = _yardstick(torch, dev, (qx, sfx, qw, sfw, lambda: fp8mm.mxfp8_gemm(qx, sfx, qw, sfw, c, workspace=gws)))
 
     rows = None
     if rank == 0 and not args.no_rows:

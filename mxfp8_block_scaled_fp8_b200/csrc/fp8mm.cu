@@ -132,25 +132,6 @@ static fp8mm_status make_sf_map(CUtensorMap* map, const void* sf, int64_t k, int
   return FP8MM_OK;
 }
 
-// 4-D map over the same scale layout with a replica dimension of stride 0:
-// uint32 [n_rt][4][n_kc][128]; box = 2 row tiles x 4 replicas x 1 K group x
-// 128 words lands in shared memory as chunk 0 four times, then chunk 1 four
-// times (4 KB); zero fill past the last row tile.
-static fp8mm_status make_sf_rep_map(CUtensorMap* map, const void* sf, int64_t k, int64_t rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
-  const int64_t n_kc = (k + 127) / 128, n_rt = (rows + 127) / 128;
-  cuuint64_t dims[4] = {128u, static_cast<cuuint64_t>(n_kc), 4u, static_cast<cuuint64_t>(n_rt)};
-  cuuint64_t strides[3] = {512u, 0u, static_cast<cuuint64_t>(n_kc) * 512u};
-  cuuint32_t box[4] = {128u, 1u, 4u, 2u};
-  cuuint32_t es[4] = {1u, 1u, 1u, 1u};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<void*>(sf), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
-  return FP8MM_OK;
-}
-
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -282,7 +263,7 @@ static Tiled tiled_kind(int kind, int64_t m, int64_t n, int64_t sms) {
 }
 
 using P1 = PairCfg<false, 6, 2>;
-using P2 = PairCfg<true, 6, 1>;
+using P2 = PairCfg<true, 5, 1>;
 
 // Largest number of co-resident 2-CTA clusters of a pair kernel (cached per
 // kernel and device).
@@ -402,7 +383,7 @@ static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uin
   if ((st = make_map(&tb, b, k, n, 128)) != FP8MM_OK) return st;
   if (mx) {
     if ((st = make_sf_map(&tsa, sfa, k, m, 1)) != FP8MM_OK) return st;
-    if ((st = make_sf_rep_map(&tsb, sfb, k, n)) != FP8MM_OK) return st;
+    if ((st = make_sf_map(&tsb, sfb, k, n, 2)) != FP8MM_OK) return st;
   } else {
     tsa = ta;  // unused in per-token mode
     tsb = tb;
@@ -429,7 +410,7 @@ static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uin
   p.group_m = pair_group_m(n, k);
   p.split = 1;
   p.dp_tiles = p.num_tiles;
-  const void* kern = mx ? reinterpret_cast<const void*>(gemm_pair_kernel<true, 6, 1>)
+  const void* kern = mx ? reinterpret_cast<const void*>(gemm_pair_kernel<true, 5, 1>)
                      : c8 ? reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2, true>)
                           : reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2>);
   const int smem = mx ? P2::kSmemBytes : P1::kSmemBytes;
@@ -459,7 +440,7 @@ static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uin
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = mx   ? cudaLaunchKernelEx(&cfg, gemm_pair_kernel<true, 6, 1>, ta, tb, tsa, tsb, p)
+  cudaError_t e = mx   ? cudaLaunchKernelEx(&cfg, gemm_pair_kernel<true, 5, 1>, ta, tb, tsa, tsb, p)
                   : c8 ? cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false, 6, 2, true>, ta, tb, tsa, tsb, p)
                        : cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false, 6, 2>, ta, tb, tsa, tsb, p);
   if (e != cudaSuccess) return cuda_fail(e);

@@ -13,13 +13,13 @@
 //
 // Block scales (mode 2): each CTA loads its A scale chunk and both B scale
 // chunks (every CTA needs all 256 B rows' scales in its own TMEM) with the
-// same pair-completed TMA loads, the B chunks as four replicas each (one
-// load through a tensor map whose replica dimension has stride 0); the MMA
-// thread copies them into the stage's TMEM columns right before that stage's
-// MMAs: A with one 32x128b.warpx4 copy, both B chunks with one 128x256b copy
-// from the replicas.  Each tcgen05.cp costs about the same tensor-pipe time
-// whatever its size, so two copies per K slab instead of three save ~6 % of
-// the kernel's cycles.
+// same pair-completed TMA loads; the MMA warp copies them into the stage's
+// TMEM columns right before that stage's MMAs, three 32x128b.warpx4 copies
+// (A, B rows 0-127, B rows 128-255).  Issued from a converged warp the copies
+// cost little (see elect_one_sync); from a lone lane each stalled the tensor
+// pipe, and B's two chunks then went as four replicas each through one
+// 128x256b copy.  Measured on B200 (8192 x 22016 x 8192, converged issue):
+// plain chunks and 5 stages are 1.3 % faster than replicas and 6 stages.
 // Moving the copies to other warps (tcgen05.st from four scale warps, or the
 // copies issued by a second thread) measured no faster, and cluster-scope
 // release arrivals from those warps made the kernel ~45 % slower.
@@ -61,7 +61,7 @@ struct PairCfg {
   static constexpr int kABytes = 128 * kBK;          // this CTA's half of A
   static constexpr int kBBytes = 128 * kBK;          // this CTA's half of B
   static constexpr int kSfaBytes = kMX ? 512 : 0;    // this CTA's 128 A rows x 4 blocks
-  static constexpr int kSfbBytes = kMX ? 4096 : 0;   // all 256 B rows x 4 blocks, two chunks x 4 replicas
+  static constexpr int kSfbBytes = kMX ? 1024 : 0;   // all 256 B rows x 4 blocks: two 512-byte chunks
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kStages * kABytes;
   static constexpr int kOffSfa = kOffB + kStages * kBBytes;
@@ -113,9 +113,9 @@ __device__ __forceinline__ void pair_unit(int u, const GemmArgs& p, int& t, int&
 constexpr int kPairPartFloats = 16 * 2 * 32 * 32;
 
 // GemmArgs fields as in gemm.cuh, with tiles_m = ceil(m/256), tiles_n =
-// ceil(n/256).  tmSFA: 3-D map over the scale layout viewed as uint32
-// [n_rt][n_kc][128]; tmSFB: 4-D map [n_rt][4 replicas, stride 0][n_kc][128]
-// (both unused in per-token mode).
+// ceil(n/256).  tmSFA, tmSFB: 3-D maps over the scale layout viewed as uint32
+// [n_rt][n_kc][128], boxes of one and two 128-row chunks (both unused in
+// per-token mode).
 template <bool kMX, int kStages, int kAccStages, bool kOut8 = false>
 __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -196,8 +196,8 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
             tma_load_2d_pair(smem + Cfg::kOffB + stage * Cfg::kBBytes, &tmB, fb, kb * kBK, nb * 256 + rank * 128);
             if constexpr (kMX) {
               tma_load_3d_pair(smem + Cfg::kOffSfa + stage * Cfg::kSfaBytes, &tmSFA, fb, 0, kb, mb * 2 + rank);
-              // both B chunks, four replicas each, in one load (a zero-stride replica dimension)
-              tma_load_4d_pair(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes, &tmSFB, fb, 0, kb, 0, nb * 2);
+              // both 128-row chunks of B's scales for this K slab in one load
+              tma_load_3d_pair(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes, &tmSFB, fb, 0, kb, nb * 2);
             }
           }
           __syncwarp();
@@ -250,8 +250,10 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
               const uint32_t sfa_t = tmem_base + static_cast<uint32_t>(Cfg::kSfCol0 + stage * Cfg::kSfColsPerStage);
               tmem_cp_32x128b_warpx4_pair(sfa_t,
                                           sf_chunk_desc(smem_u32(smem + Cfg::kOffSfa + stage * Cfg::kSfaBytes)));
-              tmem_cp_128x256b_pair(sfa_t + 8u,
-                                    sf_replicated_desc(smem_u32(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes), 2048u));
+              tmem_cp_32x128b_warpx4_pair(sfa_t + 8u,
+                                          sf_chunk_desc(smem_u32(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes)));
+              tmem_cp_32x128b_warpx4_pair(sfa_t + 12u,
+                                          sf_chunk_desc(smem_u32(smem + Cfg::kOffSfb + stage * Cfg::kSfbBytes + 512)));
 #pragma unroll
               for (int kk = 0; kk < kBK / kMmaK; ++kk)
                 mma_mxf8f6f4_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc_mxf8f6f4(256, 256, kk, kk), sfa_t,

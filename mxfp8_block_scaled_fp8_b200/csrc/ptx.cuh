@@ -317,16 +317,6 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster_addr), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
-// 4-D tiled TMA load of this CTA's part of a pair's operands, completing on
-// the leader CTA's barrier (no multicast).
-__device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* map, uint32_t mbar_cluster_addr,
-                                                 int32_t x, int32_t y, int32_t z, int32_t w) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster_addr), "r"(x), "r"(y), "r"(z), "r"(w)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
                "r"(ncols)
@@ -365,12 +355,6 @@ __device__ __forceinline__ void mma_mxf8f6f4_pair(uint32_t d_tmem, uint64_t ades
           "r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
       : "memory");
-}
-// 128 lanes x 32 bytes shared -> TMEM (8 columns) in both CTAs of the pair;
-// lane L reads bytes [0, 16) and [16, 32) from the two 16-byte core-matrix
-// columns at desc start + (L / 8) * SBO + (L % 8) * 16 and that + LBO.
-__device__ __forceinline__ void tmem_cp_128x256b_pair(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 // Scale-chunk copy shared -> TMEM performed in both CTAs of the pair, each
 // from its own shared memory at the same offset.
@@ -431,19 +415,6 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
 __device__ __forceinline__ uint64_t sf_chunk_desc(uint32_t smem_addr) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
-  d |= static_cast<uint64_t>(128u >> 4) << 32;
-  d |= static_cast<uint64_t>(1u) << 46;
-  return d;
-}
-// Descriptor of two scale chunks stored as four replicas each, chunk c's
-// replica w at c * lbo + w * 512: with SBO = 128 B, lanes 32w..32w+31 read
-// replica w line by line, so a 128x256b copy puts chunk 0 in columns 0-3 and
-// chunk 1 in columns 4-7 of every lane quarter -- the image two 32x128b.warpx4
-// copies of the chunks would make.
-__device__ __forceinline__ uint64_t sf_replicated_desc(uint32_t smem_addr, uint32_t lbo) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
-  d |= static_cast<uint64_t>((lbo & 0x3FFFFu) >> 4) << 16;
   d |= static_cast<uint64_t>(128u >> 4) << 32;
   d |= static_cast<uint64_t>(1u) << 46;
   return d;
