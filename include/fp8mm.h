@@ -95,7 +95,8 @@ typedef struct fp8mm_opts {
    * two accumulators in both scale modes). */
   int32_t kernel;
   /* Number of CTAs for the small-M kernel's stream-K split (0 = automatic:
-   * one per SM, but at least 4 K slabs of 128 per CTA). */
+   * one or two per SM, at least 4 K slabs of 128 per CTA, replaced by a
+   * tile-aligned count with s dividing the K slabs where one comes close). */
   int32_t small_m_ctas;
   /* FP8MM_FLAG_* bits. */
   uint32_t flags;
@@ -110,7 +111,9 @@ typedef struct fp8mm_opts {
  * quantized at load time); never when the preceding kernel writes them. */
 #define FP8MM_FLAG_WEIGHTS_READY 1u
 /* The small-M kernel reduces a split whose CTA count is tile-aligned (s CTAs
- * per 128-row weight tile, 2 <= s <= 8, s dividing ceil(k / 128)) inside
+ * per 128-row weight tile, 2 <= s <= min(8, ceil(k / 128)); CTA r of a tile
+ * takes K slabs [floor(r * nk / s), floor((r + 1) * nk / s)), nk = ceil(k /
+ * 128)) inside
  * thread-block clusters of s CTAs, through distributed shared memory, and
  * then needs no workspace.  With this flag it reduces such splits through
  * the workspace instead (identical results; for comparison and testing). */

@@ -493,12 +493,14 @@ static fp8mm_status launch_small_m_t(const CUtensorMap& tw, const CUtensorMap& t
 constexpr int64_t kMaxClusterSplit = 8;
 
 // CTAs per weight tile when `ctas` is a tile-aligned split that the kernel can
-// reduce inside clusters (2..8 CTAs per tile, dividing the tile's K slabs);
-// 0 otherwise.
+// reduce inside clusters (2..8 CTAs per tile, each with at least one K slab);
+// 0 otherwise.  CTA b = t*s + r owns slabs [floor(b*U/G), floor((b+1)*U/G))
+// = t*num_k + [floor(r*num_k/s), floor((r+1)*num_k/s)): always inside tile t,
+// whether or not s divides num_k.
 static int cluster_split(int64_t ctas, int64_t n_tiles, int64_t num_k) {
   if (ctas % n_tiles != 0) return 0;
   const int64_t s = ctas / n_tiles;
-  return (s >= 2 && s <= kMaxClusterSplit && num_k % s == 0) ? static_cast<int>(s) : 0;
+  return (s >= 2 && s <= kMaxClusterSplit && s <= num_k) ? static_cast<int>(s) : 0;
 }
 
 // Largest tile-aligned CTA count (s CTAs per tile, 2 <= s <= 8, s dividing
@@ -528,17 +530,20 @@ static int small_m_l2_ahead(int64_t units, int64_t ctas, int64_t sms) {
 // with s dividing the tile's K slabs, so every CTA runs one segment inside
 // one tile and all contributors of a tile are equal (and reduce inside a
 // cluster) -- when the largest such count that fits two CTAs per SM comes
-// within 80 % of it (16-token tiles) or 60 % (larger tiles, whose split-tile
+// within 75 % of it (16-token tiles) or 60 % (larger tiles, whose split-tile
 // partials cost more).  Measured on B200 with back-to-back calls (GEMM alone,
 // before 48- and 64-token tiles ran two per SM): 6144 x
 // 4096 at m <= 32 with 192 CTAs instead of 148 is 12-17 % faster and at m = 64
 // with 96 instead of 148 10 %, 4096 x 14336 at m <= 8 with 256 instead of 148
 // 8 % and at m = 64 with 128 instead of 148 6 %, 14336 x 4096 at m = 32 with
-// 224 instead of 296 5 % and at m = 64 with 112 instead of 148 9 %; at m <= 8
-// there 224 is 3 % slower than 296 (more bytes in flight outweigh the
-// alignment for 16-token tiles).  Counts between the aligned ones are slower
-// than both neighbours (e.g. 6144 x 4096, m = 1: 8.5 us at 192 CTAs, 9.6-10.4
-// us at 160-240).
+// 224 instead of 296 5 % and at m = 64 with 112 instead of 148 9 %.  With
+// converged issue (see elect_one_sync), 14336 x 4096 at m <= 16 with 224
+// instead of 296 is 4-5 % faster (13.3 against 13.9 us; it was 3 % slower
+// before).  Splits that do not divide the K slabs (cluster_split allows them)
+// measured slower than the dividing ones next to them (6144 x 4096: 144 and
+// 240 CTAs 8.8 us against 7.9 us at 192; 4096 x 14336: 160-224 against 128
+// and 256).  Counts between the aligned ones are slower than both neighbours
+// (e.g. 6144 x 4096, m = 1: 8.5 us at 192 CTAs, 9.6-10.4 us at 160-240).
 constexpr int64_t kMinSlabsPerCta = 4;
 static int64_t best_cluster_ctas(int64_t n_tiles, int64_t num_k, int64_t slots) {
   int64_t best = 0;
@@ -555,7 +560,7 @@ static int small_m_ctas(int64_t units, int64_t n_tiles, int64_t num_k, int nm, i
     int64_t aligned = 0;
     for (int64_t s = 1; s <= num_k / kMinSlabsPerCta; ++s)
       if (num_k % s == 0 && n_tiles * s <= slots) aligned = n_tiles * s;
-    if (aligned > 0 && aligned * 10 >= g * (nm <= 16 ? 8 : 6)) g = aligned;
+    if (aligned > 0 && aligned * 20 >= g * (nm <= 16 ? 15 : 12)) g = aligned;
   }
   g = std::min<int64_t>(g, units);
   return static_cast<int>(std::max<int64_t>(g, 1));

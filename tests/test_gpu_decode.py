@@ -157,12 +157,15 @@ N_TILES = {name: -(-n // 128) for name, (n, k) in synthetic.DECODE_SHAPES.items(
 
 
 @pytest.mark.parametrize("name,m,s", [("qkv", 1, 4), ("qkv", 64, 2), ("up", 8, 2), ("up", 32, 4), ("up", 64, 8),
-                                      ("down", 1, 8), ("down", 16, 7), ("down", 48, 4), ("down", 64, 2)])
+                                      ("down", 1, 8), ("down", 16, 7), ("down", 48, 4), ("down", 64, 2),
+                                      ("qkv", 1, 3), ("qkv", 16, 5), ("qkv", 64, 6), ("up", 1, 3),
+                                      ("down", 8, 3), ("down", 32, 5), ("down", 64, 6)])
 def test_cluster_reduction_equals_workspace_reduction(decode_data, name, m, s):
-    """s CTAs per weight tile (2 <= s <= 8, s dividing the tile's K slabs:
-    32 for up and qkv, 112 for down) are reduced inside a cluster through
-    distributed shared memory; the same partition reduced through the
-    workspace gives identical bits, and both meet the bar."""
+    """s CTAs per weight tile (2 <= s <= 8; the tile's K slabs -- 32 for up
+    and qkv, 112 for down -- split as floor(r*num_k/s), so s need not divide
+    them) are reduced inside a cluster through distributed shared memory; the
+    same partition reduced through the workspace gives identical bits, and
+    both meet the bar."""
     import oracle as orc
     weights, xs = decode_data
     qw, sfw, gw, gsfw = weights[name]
@@ -186,10 +189,12 @@ def test_cluster_reduction_equals_workspace_reduction(decode_data, name, m, s):
     assert fp8mm.last_device_error() == 0
 
 
-@pytest.mark.parametrize("m,n,k,s", [(5, 200, 512, 2), (17, 130, 4096, 8), (40, 384, 896, 7), (64, 257, 1024, 4)])
+@pytest.mark.parametrize("m,n,k,s", [(5, 200, 512, 2), (17, 130, 4096, 8), (40, 384, 896, 7), (64, 257, 1024, 4),
+                                     (9, 300, 896, 5), (33, 140, 640, 3), (2, 129, 768, 6)])
 def test_cluster_reduction_ragged(m, n, k, s):
     """Ragged weight tiles (n not a multiple of 128) and token counts that fill
-    part of the 16/32/48/64-token tile, with 2, 4, 7 and 8 CTAs per tile."""
+    part of the 16/32/48/64-token tile, with 2..8 CTAs per tile, some of which
+    do not divide the tile's K slabs (7 slabs in 5 parts, 5 in 3, 6 in 6)."""
     import oracle as orc
     x = synthetic.random_bf16((m, k), seed=m * 7 + k)
     w = synthetic.random_bf16((n, k), seed=n * 11 + k, sigma=0.02)
