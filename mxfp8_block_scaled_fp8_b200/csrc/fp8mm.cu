@@ -195,8 +195,7 @@ static fp8mm_status launch_tiled_kernel(Kern kern, int grid, const CUtensorMap& 
                                         const GemmArgs& p, cudaStream_t stream, int dev) {
   fp8mm_status st = ensure_smem(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes, dev);
   if (st != FP8MM_OK) return st;
-  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, stream>>>(ta, tb, p);
-  return launched();
+  return launch_pdl(kern, dim3(grid), dim3(kGemmThreads), Cfg::kSmemBytes, stream, ta, tb, p);
 }
 
 // Single-SM tiled kernel, 128 x 256 tiles or (n128) 128 x 128 tiles.
@@ -429,17 +428,19 @@ static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uin
   }
   pairs = std::min(pairs, p.dp_tiles + (p.num_tiles - p.dp_tiles) * p.split);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see the kernel's griddep calls
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = mx   ? cudaLaunchKernelEx(&cfg, gemm_pair_kernel<true, 5, 1>, ta, tb, tsa, tsb, p)
                   : c8 ? cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false, 6, 2, true>, ta, tb, tsa, tsb, p)
                        : cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false, 6, 2>, ta, tb, tsa, tsb, p);

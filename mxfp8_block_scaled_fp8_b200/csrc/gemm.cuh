@@ -187,6 +187,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Launched with programmatic stream serialisation: the set-up below may
+  // overlap the preceding kernel; the producer and the epilogue wait for it
+  // before their first global access.
+  griddep_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -217,6 +221,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     // The whole warp runs the loop; one elected lane issues (see elect_one_sync).
+    griddep_wait();  // A, B and their scales may be written by the preceding kernel
     {
       int stage = 0;
       uint32_t phase = 0;
@@ -330,6 +335,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // its kBN/2 accumulator values into registers with kBN/64 loads and a
     // single wait, then releases the accumulator at once, so the next tile's
     // MMAs overlap the scaling, conversion and stores below.
+    griddep_wait();  // C and the scales may belong to the preceding kernel
     const int sp = warp & 3;
     const int col_half = (warp - 2) >> 2;
     constexpr int kHalf = kBN / 2;

@@ -141,6 +141,11 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
   const bool leader = (rank == 0);
   const int pair = static_cast<int>(cluster_id_x());
   const int npairs = static_cast<int>(num_clusters_x());
+  // Launched with programmatic stream serialisation: the set-up below may
+  // overlap the preceding kernel; the producer and the epilogue wait for it
+  // before their first global access, and a following kernel may start its own
+  // set-up as SMs free up.
+  griddep_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -176,6 +181,7 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer (both CTAs)
     // The whole warp runs the loop; one elected lane issues (see elect_one_sync).
+    griddep_wait();  // A, B and their scales may be written by the preceding kernel
     {
       int stage = 0;
       uint32_t phase = 0, issued_mask = 0, issued_parity = 0;
@@ -287,6 +293,7 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
     __syncwarp();
   } else {
     // ------------------------------------------------------ epilogue (both CTAs)
+    griddep_wait();  // C, the workspace and the scales may belong to the preceding kernel
     const int sp = warp & 3;
     const int quarter = (warp - Cfg::kEpiWarp0) >> 2;  // 64-column slice of the 256-column tile
     float s_out = 1.f, r_out = 1.f;
