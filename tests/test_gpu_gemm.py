@@ -350,6 +350,32 @@ def test_attn_rowwise_full():
     assert fp8mm.last_device_error() == 0
 
 
+def test_tail_split_e4m3_out():
+    """The E4M3-output GEMM with the last wave split along K (2560 x 2048 x 8192: 80 tiles, 6 in 4 parts
+    with 74 pairs): every code equals or neighbours the unsplit result's (same accumulator up to summation
+    order), a second call is identical and the counters are back at zero."""
+    import oracle as orc
+    m, n, k = 2560, 2048, 8192
+    a = synthetic.random_bf16((m, k), seed=81)
+    bt = synthetic.random_bf16((n, k), seed=82, sigma=0.05)
+    ga, gsa = fp8mm.fp8_quantize_rowwise(gu.to_dev(a))
+    gb, gsb = fp8mm.fp8_quantize_rowwise(gu.to_dev(bt))
+    so = torch.tensor([0.25], dtype=torch.float32, device="cuda")
+    ws = _ws(m, n, k)
+    c_split = fp8mm.fp8_gemm_e4m3_out(ga, gb, gsa, gsb, so, workspace=ws)
+    c_again = fp8mm.fp8_gemm_e4m3_out(ga, gb, gsa, gsb, so, workspace=ws)
+    c_plain = fp8mm.fp8_gemm_e4m3_out(ga, gb, gsa, gsb, so)
+    torch.cuda.synchronize()
+    assert torch.equal(c_split, c_again)
+    assert not ws[-256:].any()
+    dec = orc.e4m3_decode_table()
+    x, y = dec[c_split.cpu().numpy()], dec[c_plain.cpu().numpy()]
+    lo, hi = np.minimum(x, y), np.maximum(x, y)
+    codes = np.sort(np.unique(dec[np.isfinite(dec)]))
+    assert np.all(np.searchsorted(codes, hi) - np.searchsorted(codes, lo) <= 1)
+    assert fp8mm.last_device_error() == 0
+
+
 def _tiles_equal(c1, c2):
     """Per 256 x 256 output tile: whether the two results are bit-identical there."""
     m, n = c1.shape
