@@ -59,6 +59,7 @@ struct GemmArgs {
   int dp_tiles;              // paired-SM kernel: tiles [0, dp_tiles) run whole, the rest in split parts
   float* partials;           // split > 1: fp32 partials [(num_tiles - dp_tiles) * split][2][128 * 256]
   unsigned* tickets;         // split > 1: arrivals per (split tile, CTA rank), zero between calls
+  int tma_c;                 // paired MX kernel: whole tiles' C goes out by TMA stores through shared memory
 };
 
 // Per-token / per-channel scaling of an fp32 accumulator, sa * sb * acc

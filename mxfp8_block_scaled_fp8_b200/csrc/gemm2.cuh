@@ -70,7 +70,11 @@ struct PairCfg {
   // full, empty per stage; acc_full, acc_empty per accumulator; drain; epi_sync
   static constexpr int kNumBars = 2 * kStages + 2 * kAccStages + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  // MX: one 2 KiB staging buffer per epilogue warp (32 rows x 32 bf16 with the
+  // 64-byte swizzle) for the TMA stores of C.
+  static constexpr int kEpiBufBytes = 2048;
+  static constexpr int kOffEpi = kMX ? ((kOffMisc + 16 + 1023) / 1024) * 1024 : kOffMisc + 16;
+  static constexpr int kSmemBytes = kOffEpi + (kMX ? 16 * kEpiBufBytes : 0) + 1024;
   // bytes of both CTAs' loads, all completing on the leader's barrier
   static constexpr uint32_t kTxPair = 2u * (kABytes + kBBytes + kSfaBytes + kSfbBytes);
   static constexpr int kSfColsPerStage = 16;                       // A: columns 0-3, B: 8-15
@@ -115,12 +119,13 @@ constexpr int kPairPartFloats = 16 * 2 * 32 * 32;
 // GemmArgs fields as in gemm.cuh, with tiles_m = ceil(m/256), tiles_n =
 // ceil(n/256).  tmSFA, tmSFB: 3-D maps over the scale layout viewed as uint32
 // [n_rt][n_kc][128], boxes of one and two 128-row chunks (both unused in
-// per-token mode).
+// per-token mode).  tmC (MX mode with p.tma_c): C as bf16 [m][n] with row
+// stride ldc, box 32 x 32, 64-byte swizzle; stores past m or n are clipped.
 template <bool kMX, int kStages, int kAccStages, bool kOut8 = false>
 __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                     const GemmArgs p) {
+                     const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
   using Cfg = PairCfg<kMX, kStages, kAccStages>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -384,6 +389,37 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
         if (threadIdx.x == Cfg::kEpiWarp0 * 32) *ticket = 0u;
         continue;
       }
+      if (kMX && p.tma_c) {
+        // bf16 rows into the warp's staging buffer (lane = row; 16-byte chunk q
+        // of a 64-byte row lands at chunk q ^ ((row >> 1) & 3), the 64-byte
+        // swizzle, so each 16-byte store of the warp takes four wavefronts),
+        // then one TMA store of the 32 x 32 block.  Measured on B200 (ffn_up):
+        // 0.8 % faster than the 32-byte stores from registers, bit-identical.
+        uint8_t* buf = smem + Cfg::kOffEpi + wl * Cfg::kEpiBufBytes;
+        const int row0 = mb * 256 + static_cast<int>(rank) * 128 + sp * 32;
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[ch][2 * j]), __uint_as_float(r[ch][2 * j + 1]));
+            packed[j] = *reinterpret_cast<uint32_t*>(&h);
+          }
+          if (lane == 0) bulk_wait_read0();  // the previous store from this buffer has read it
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(buf + lane * 64 + ((q ^ ((lane >> 1) & 3)) * 16)) =
+                make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, buf, nb * 256 + quarter * 64 + ch * 32, row0);
+            bulk_commit();
+          }
+        }
+        continue;
+      }
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         const int col0 = nb * 256 + quarter * 64 + ch * 32;
@@ -398,6 +434,7 @@ __global__ void __launch_bounds__(PairCfg<kMX, kStages, kAccStages>::kThreads, 1
         store_out32<kOut8>(p, row, col0, v, s_out, r_out, out_fast);
       }
     }
+    if (kMX && p.tma_c && lane == 0) bulk_wait_all0();  // this warp's stores of C are complete
   }
 
   tc_fence_before();

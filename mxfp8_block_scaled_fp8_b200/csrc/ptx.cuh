@@ -100,6 +100,20 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 }
 
 // ------------------------------------------------------------ async copies
+// 2-D tiled TMA store shared -> global in a bulk async-group (no multicast).
+// x is the innermost coordinate in elements; callers keep x * element size a
+// multiple of 16 bytes and never start a store at a negative coordinate.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the calling thread's bulk stores have read their shared memory
+// (read0) or have completed (all0).
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
