@@ -134,18 +134,18 @@ static fp8mm_status make_sf_map(CUtensorMap* map, const void* sf, int64_t k, int
 
 // 2-D map over a bf16 output C [m][n] with row stride ldc elements, for the
 // paired MX kernel's TMA stores: box 32 columns x 32 rows, 64-byte swizzle.
-// Needs a 16-byte aligned base and ldc * 2 a multiple of 16.
-static fp8mm_status make_c_map(CUtensorMap* map, void* c, int64_t m, int64_t n, int64_t ldc) {
+// Needs a 16-byte aligned base and ldc * 2 a multiple of 16.  An optional
+// fast path: false (and no error recorded) when the map cannot be made.
+static bool make_c_map(CUtensorMap* map, void* c, int64_t m, int64_t n, int64_t ldc) {
   EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
+  if (fn == nullptr) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(m)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldc) * 2u};
   cuuint32_t box[2] = {32u, 32u};
   cuuint32_t es[2] = {1u, 1u};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
-  return FP8MM_OK;
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
 }
 
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -429,9 +429,7 @@ static fp8mm_status launch_pair(bool mx, const void* a, const void* b, const uin
   // (16-byte aligned base and row stride); otherwise, and for split tiles, by
   // stores from registers.
   tc = ta;  // unused unless p.tma_c
-  p.tma_c = (mx && c != nullptr && aligned(c, 16) && (ldc * 2) % 16 == 0 && make_c_map(&tc, c, m, n, ldc) == FP8MM_OK)
-                ? 1
-                : 0;
+  p.tma_c = (mx && c != nullptr && aligned(c, 16) && (ldc * 2) % 16 == 0 && make_c_map(&tc, c, m, n, ldc)) ? 1 : 0;
   const void* kern = mx ? reinterpret_cast<const void*>(gemm_pair_kernel<true, 5, 1>)
                      : c8 ? reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2, true>)
                           : reinterpret_cast<const void*>(gemm_pair_kernel<false, 6, 2>);
