@@ -15,9 +15,10 @@
 // resets the counter.  No CTA ever waits for another.
 //
 // With kCR (cluster reduction) the CTA count is tile-aligned: s = G / n_tiles
-// CTAs per weight tile, s dividing the tile's K slabs, so CTA b runs the one
-// segment b % s of tile b / s, and the s contributors of a tile are launched
-// as one thread-block cluster.  Each writes its fp32 partial into its own
+// CTAs per weight tile (s need not divide the tile's K slabs: CTA b = t*s + r
+// owns slabs [floor(r*num_k/s), floor((r+1)*num_k/s)) of tile t), so CTA b
+// runs the one segment b % s of tile b / s, and the s contributors of a tile
+// are launched as one thread-block cluster.  Each writes its fp32 partial into its own
 // (idle) weight ring, signals every peer's mbarrier, and then sums the slice
 // of weight rows [r*128/s, (r+1)*128/s) that its rank r owns over all s
 // partials, read through distributed shared memory in rank order (the same

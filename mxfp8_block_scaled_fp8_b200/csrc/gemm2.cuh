@@ -5,8 +5,9 @@
 // for the block-scaled mode), computed by 2-CTA clusters on 256 x 256 output
 // tiles.  Each CTA of a pair loads its own 128-row half of the A tile and its
 // own 128-row half of the B tile; nothing is multicast.  Those loads complete
-// on the rank-0 CTA's barrier, whose one thread issues the cta_group::2 MMAs
-// (M = 256, N = 256, K = 32) that read A and B from both CTAs' shared memory
+// on the rank-0 CTA's barrier, whose MMA warp issues (from one elected lane)
+// the cta_group::2 MMAs (M = 256, N = 256, K = 32) that read A and B from both
+// CTAs' shared memory
 // and accumulate 128 rows in each CTA's TMEM.  Per 128-byte K slab a CTA moves
 // 32 KiB into shared memory for 128x256x128 MACs, two thirds of what the
 // single-CTA 128x256 tile needs.
