@@ -28,6 +28,13 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  All work is enqueued asynchronously on it.  No call syncs the
  *     host, except fp8mm_last_device_error and fp8mm_selftest_wait_timeout.
+ *   - Every kernel is launched with programmatic stream serialisation: it may
+ *     begin (set-up, and for the small-M kernel under
+ *     FP8MM_FLAG_WEIGHTS_READY the weight stream) while the preceding kernel
+ *     on the stream finishes, and waits for it in-kernel
+ *     (griddepcontrol.wait) before it reads an input or writes an output
+ *     that kernel may use.  Stream order is therefore kept as for ordinary
+ *     launches.
  *   - Matrices are row-major.  A is [m, k] and B is given as [n, k] (the
  *     transpose of the pages' logical [k, n], K contiguous -- the "weight_t"
  *     layout of the mm_mxfp8 call).  C is [m, n] bf16 with row stride ldc
