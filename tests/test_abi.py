@@ -4,6 +4,8 @@ layout helpers agree with the layout formula the header documents."""
 import ctypes
 import os
 import re
+import shutil
+import subprocess
 
 import numpy as np
 import pytest
@@ -215,3 +217,22 @@ def test_pair_split_plan():
     assert plan(64, 4096, 8192, 74) == (1, 16)           # m <= 64: the small-M kernel's business
     assert plan(8192, 22016, 8192, 72) == (4, 2736)      # 72 pairs: 38 waves + 16; 72 // 16 = 4
     assert plan(0, 128, 128, 74) == (1, 0)
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="gcc not available")
+def test_opts_struct_layout_matches_the_header(tmp_path):
+    """The binding's ctypes fp8mm_opts has the header's size and field offsets (compiled with gcc from
+    include/fp8mm.h), so the options a Python caller sets are the ones the library reads."""
+    src = tmp_path / "layout.c"
+    fields = [name for name, _ in binding.Opts._fields_]
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "fp8mm.h"\nint main(void) {\n'
+                   '  printf("size %zu\\n", sizeof(fp8mm_opts));\n'
+                   + "".join(f'  printf("{f} %zu\\n", offsetof(fp8mm_opts, {f}));\n' for f in fields)
+                   + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                        check=True).stdout.splitlines())
+    assert int(out["size"]) == ctypes.sizeof(binding.Opts)
+    for f in fields:
+        assert int(out[f]) == getattr(binding.Opts, f).offset, f
